@@ -1,0 +1,301 @@
+/*
+ * nvfp4_oracle.c -- plain, slow CPU reference for the NVFP4 W4A4 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file; only the tests, the smoke check and the benchmark's CPU-baseline leg
+ * do.  It shares no code, header, table or constant generator with the CUDA
+ * library.
+ *
+ * What it follows:
+ *  - "Why Gated DeltaNet Survives 4-Bit Quantization", §2 "NVFP4": values are
+ *    E2M1 (4 bits), one E4M3 scale per 16-element block set to blockmax/6, one
+ *    FP32 scale per tensor; W4A4 quantizes weights and activations alike and the
+ *    GEMM consumes both.
+ *  - same paper, §5 intro: "fake quantization" (quantize, dequantize, continue in
+ *    high precision) -- the GEMM below dequantizes and accumulates in fp64.
+ *  - same paper, §6 "Per-module calibration vs. fused-GEMM scaling": each module
+ *    of a fused GEMM keeps its own FP32 global scale; collapsing them to the
+ *    maximum without touching the block scales is the mismatch that paragraph
+ *    describes (kept here only as a negative control).
+ *  - "Gemma-4-31B-IT-NVFP4-FP8attn-text" model card, §Verification: the stored
+ *    per-tensor scale satisfies max(block scale) x global x 6 = absmax, 6 being
+ *    the largest E2M1 magnitude, so the global scale is the dequantization
+ *    multiplier absmax / (6 * 448); §Limitations: packed uint8 holding two codes
+ *    per byte along the input dimension.
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *  R1  amax is the exact max |x| over the tensor (segment) in fp32.
+ *  R2  s = amax / 2688 in fp32 round-to-nearest (2688 = 6 * 448).
+ *  R4  d_g = s * 6 (fp32); sb_f = min(bmax / d_g, 448) (fp32); d_g == 0 -> sb_f = 0.
+ *  R5  sb = E4M3(sb_f): nearest E4M3 (FN, bias 7, subnormals kept, max 448)
+ *      value, ties to the even code, saturating at 448 (0x7E); never 0x7F.
+ *  R6  sd = value(sb); d = sd * s (fp32); r = 0 if d == 0 else min(1/d, FLT_MAX).
+ *  R7  v = x * r (fp32); code = E2M1(v): nearest grid value, ties to the even
+ *      code, |v| beyond 6 saturates to 6; the sign bit is the sign of v, so
+ *      negative values that round to zero encode as 0x8.
+ *  R9  byte j of a packed row holds code(2j) in bits 0..3 and code(2j+1) in
+ *      bits 4..7.
+ *  R10 physical scale layout consumed by the tensor cores: rows padded to 128,
+ *      scale columns padded to 4; 512-byte atoms of 128 rows x 4 scale columns,
+ *      atoms ordered K-fastest; inside an atom byte (r%32)*16 + ((r%128)/32)*4 + c%4.
+ *      Pad bytes are 0.
+ *  R11 GEMM: exact fp64 sum over k of value(code_x)*sd_x * value(code_w)*sd_w,
+ *      then times s_x and times s_w of the column's segment, in fp64.
+ *
+ * Build: gcc -O2 -fopenmp -fPIC -shared -ffp-contract=off -fno-fast-math
+ */
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* Number formats                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa.
+ * Exponent field 0 is subnormal: 0.m x 2^0 = m/2.  Magnitudes 0,0.5,1,1.5,2,3,4,6. */
+double or_e2m1_value(uint32_t code)
+{
+    uint32_t sign = (code >> 3) & 1u, e = (code >> 1) & 3u, m = code & 1u;
+    double mag;
+    if (e == 0)
+        mag = 0.5 * (double)m;
+    else
+        mag = ldexp(1.0 + 0.5 * (double)m, (int)e - 1);
+    return sign ? -mag : mag;
+}
+
+/* E4M3, "FN" flavour: bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0 mantissa.
+ * No infinities; exponent 15 with mantissa 7 is NaN; largest finite 448 (0x7E).
+ * Exponent field 0 is subnormal: m/8 x 2^-6. */
+double or_e4m3_value(uint32_t code)
+{
+    uint32_t sign = (code >> 7) & 1u, e = (code >> 3) & 15u, m = code & 7u;
+    double mag;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, (int)e - 7);
+    return sign ? -mag : mag;
+}
+
+/* Index of the representable magnitude nearest to a >= 0 among codes
+ * 0..ncodes-1 (ascending values); a tie goes to the even code; anything past
+ * the last value is that last value (saturation). */
+static uint32_t nearest_code(double a, double (*value)(uint32_t), uint32_t ncodes)
+{
+    double top = value(ncodes - 1);
+    if (!(a <= top))
+        return ncodes - 1;
+    uint32_t best = 0;
+    double best_dist = fabs(a - value(0));
+    for (uint32_t c = 1; c < ncodes; ++c) {
+        double dist = fabs(a - value(c));
+        if (dist < best_dist || (dist == best_dist && (c & 1u) == 0)) {
+            best = c;
+            best_dist = dist;
+        }
+    }
+    return best;
+}
+
+/* E2M1 encode with round-to-nearest-even and saturation at 6 (R7). */
+uint32_t or_e2m1_encode(float v)
+{
+    uint32_t sign = signbit(v) ? 8u : 0u;
+    return sign | nearest_code(fabs((double)v), or_e2m1_value, 8);
+}
+
+/* E4M3 encode of a non-negative scale with round-to-nearest-even and
+ * saturation at 448 (R5); the 127 finite non-negative codes are searched. */
+uint32_t or_e4m3_encode(float v)
+{
+    uint32_t sign = signbit(v) ? 0x80u : 0u;
+    return sign | nearest_code(fabs((double)v), or_e4m3_value, 127);
+}
+
+float or_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Scales                                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* R1: max |x| over rows [r0, r1) of a bf16 matrix with row stride ld. */
+float or_amax_bf16(const uint16_t *x, int64_t r0, int64_t r1, int64_t k, int64_t ld)
+{
+    float amax = 0.0f;
+    for (int64_t r = r0; r < r1; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            float a = fabsf(or_bf16_to_f32(x[r * ld + j]));
+            if (a > amax || isnan(a))
+                amax = a;
+        }
+    return amax;
+}
+
+/* R2: per-tensor global scale, the dequantization multiplier. */
+float or_global_scale(float amax)
+{
+    float six_times_448 = 6.0f * 448.0f; /* 2688, exact */
+    return amax / six_times_448;
+}
+
+/* R4 + R5: E4M3 block scale for a block with max magnitude bmax under global s. */
+uint32_t or_block_scale(float bmax, float s)
+{
+    float d_g = s * 6.0f;
+    float sb_f = (d_g == 0.0f) ? 0.0f : bmax / d_g;
+    if (sb_f > 448.0f)
+        sb_f = 448.0f;
+    return or_e4m3_encode(sb_f);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantization of rows                                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Quantize rows of a bf16 matrix X[rows, k] (row stride ld, k % 16 == 0).
+ * row_scale[r] is the FP32 global scale of the row's tensor (segment).
+ * Outputs: q[rows, k/2] packed codes (R9), sf[rows, k/16] logical E4M3 block
+ * scales, one byte per 16-element block along k. */
+void or_quantize(const uint16_t *x, int64_t rows, int64_t k, int64_t ld, const float *row_scale,
+                 uint8_t *q, uint8_t *sf)
+{
+    const int64_t nblk = k / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const float s = row_scale[r];
+        for (int64_t b = 0; b < nblk; ++b) {
+            const uint16_t *blk = x + r * ld + b * 16;
+            float vals[16];
+            float bmax = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                vals[i] = or_bf16_to_f32(blk[i]);
+                if (fabsf(vals[i]) > bmax)
+                    bmax = fabsf(vals[i]);
+            }
+            uint32_t sb = or_block_scale(bmax, s);                  /* R4, R5 */
+            float sd = (float)or_e4m3_value(sb);
+            float d = sd * s;                                       /* R6 */
+            float rcp = 0.0f;
+            if (d != 0.0f) {
+                rcp = 1.0f / d;
+                if (rcp > FLT_MAX)
+                    rcp = FLT_MAX;
+            }
+            sf[r * nblk + b] = (uint8_t)sb;
+            for (int i = 0; i < 16; i += 2) {                       /* R7, R9 */
+                float v0 = vals[i] * rcp;
+                float v1 = vals[i + 1] * rcp;
+                uint32_t lo = or_e2m1_encode(v0), hi = or_e2m1_encode(v1);
+                q[r * (k / 2) + b * 8 + i / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+}
+
+/* Dequantize packed rows back to fp64 values (global scale included). */
+void or_dequantize(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t k, const float *row_scale,
+                   double *out)
+{
+    const int64_t nblk = k / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            uint8_t byte = q[r * (k / 2) + j / 2];
+            uint32_t code = (j & 1) ? (byte >> 4) : (byte & 15u);
+            out[r * k + j] = or_e2m1_value(code) * or_e4m3_value(sf[r * nblk + j / 16]) * (double)row_scale[r];
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Physical scale-factor layout (R10)                                        */
+/* ------------------------------------------------------------------------ */
+
+int64_t or_sf_physical_bytes(int64_t rows, int64_t k)
+{
+    int64_t rows_pad = (rows + 127) / 128 * 128;
+    int64_t cols_pad = ((k / 16) + 3) / 4 * 4;
+    return rows_pad * cols_pad;
+}
+
+int64_t or_sf_offset(int64_t r, int64_t c, int64_t k)
+{
+    int64_t cols_pad = ((k / 16) + 3) / 4 * 4;
+    int64_t atoms_per_row_block = cols_pad / 4;
+    int64_t atom = (r / 128) * atoms_per_row_block + c / 4;
+    return atom * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+}
+
+/* Scatter logical sf[rows, k/16] into the physical buffer (pads zero). */
+void or_sf_to_physical(const uint8_t *sf, int64_t rows, int64_t k, uint8_t *phys)
+{
+    memset(phys, 0, (size_t)or_sf_physical_bytes(rows, k));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < k / 16; ++c)
+            phys[or_sf_offset(r, c, k)] = sf[r * (k / 16) + c];
+}
+
+/* ------------------------------------------------------------------------ */
+/* GEMM on dequantized operands (R11)                                        */
+/* ------------------------------------------------------------------------ */
+
+/* out[i, n] (i over the nsel selected activation rows) =
+ *   sum_k deq(Qx)[rows[i], k] * deq(Qw)[n, k]  with per-operand E4M3 block scales,
+ * times s_x times col_scale[n], all in fp64.  col_scale[n] is the weight global
+ * scale of the segment that holds output column n. */
+void or_linear_rows(const uint8_t *qx, const uint8_t *sfx, float s_x, const int64_t *rows, int64_t nsel,
+                    const uint8_t *qw, const uint8_t *sfw, const float *col_scale, int64_t n, int64_t k,
+                    double *out)
+{
+    const int64_t nblk = k / 16;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)(nsel * k));
+    for (int64_t i = 0; i < nsel; ++i)
+        for (int64_t j = 0; j < k; ++j) {
+            uint8_t byte = qx[rows[i] * (k / 2) + j / 2];
+            uint32_t code = (j & 1) ? (byte >> 4) : (byte & 15u);
+            xd[i * k + j] = or_e2m1_value(code) * or_e4m3_value(sfx[rows[i] * nblk + j / 16]);
+        }
+#pragma omp parallel
+    {
+        double *wd = (double *)malloc(sizeof(double) * (size_t)k);
+#pragma omp for schedule(static)
+        for (int64_t c = 0; c < n; ++c) {
+            for (int64_t j = 0; j < k; ++j) {
+                uint8_t byte = qw[c * (k / 2) + j / 2];
+                uint32_t code = (j & 1) ? (byte >> 4) : (byte & 15u);
+                wd[j] = or_e2m1_value(code) * or_e4m3_value(sfw[c * nblk + j / 16]);
+            }
+            for (int64_t i = 0; i < nsel; ++i) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < k; ++j)
+                    acc += xd[i * k + j] * wd[j];
+                out[i * n + c] = acc * (double)s_x * (double)col_scale[c];
+            }
+        }
+        free(wd);
+    }
+    free(xd);
+}
+
+int or_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
