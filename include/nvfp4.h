@@ -1,0 +1,176 @@
+/*
+ * nvfp4.h -- C ABI of the NVFP4 W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer is Y = X . W^T with both operands in NVFP4, as described in
+ * "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4 W4A4 for the Recurrent
+ * Half of a Hybrid 27B LLM", §2 "NVFP4": values are E2M1 (4-bit), each run of 16
+ * consecutive elements along K shares one E4M3 block scale (blockmax/6), and a
+ * tensor carries one FP32 global scale.  The FP32 global scale s stored and
+ * consumed here is the dequantization multiplier, s = absmax / (6 * 448)
+ * (Gemma-4-31B-IT-NVFP4-FP8attn-text model card, §Verification:
+ * max(block scale) x s x 6 = absmax).
+ *
+ * Three steps run on the GPU:
+ *   1. activation quantization (amax -> s_x, 16-element E4M3 block scales,
+ *      E2M1 codes packed two per byte);
+ *   2. block-scaled FP4 GEMM with FP32 accumulation on the tcgen05 tensor cores;
+ *   3. an epilogue that multiplies each output column by s_x * s_w[segment]
+ *      and writes bf16.  A fused GEMM over several modules concatenated along N
+ *      keeps one weight global scale per module (segment); the paper's §6
+ *      "Per-module calibration vs. fused-GEMM scaling" shows what goes wrong
+ *      when those are collapsed to one.
+ *
+ * Conventions for every entry point
+ *   - All pointers marked "device" are CUDA device (or managed) pointers; the
+ *     caller allocates and owns every buffer, including the workspace.  The
+ *     library allocates no device memory.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  No entry point synchronizes, except
+ *     nvfp4_get_device_error().
+ *   - Arguments are validated on the host before anything is enqueued; a call
+ *     that returns an error enqueued nothing.  CUDA launch failures map to
+ *     NVFP4_ERR_CUDA (cudaGetLastError() is consumed).
+ *   - Conditions only the GPU can see (non-finite amax, a pipeline wait that
+ *     ran out) are recorded in a per-device error word, read and cleared by
+ *     nvfp4_get_device_error().
+ *
+ * Layouts
+ *   X, W    bf16, row-major, [rows, K] with a row stride (ld*) in elements;
+ *           ld* * 2 bytes and the base address must be multiples of 16.
+ *   Q       packed E2M1 codes, [rows, K/2] bytes, row stride K/2; byte j of a
+ *           row holds the code of element 2j in bits 0..3 and of element 2j+1
+ *           in bits 4..7.  Code bits: sign (bit 3), exponent (bits 2..1, bias 1),
+ *           mantissa (bit 0).
+ *   SF      E4M3 block scales in the tensor-core layout: rows padded to 128,
+ *           scale columns (K/16) padded to 4; 512-byte atoms of 128 rows x 4
+ *           scale columns, atoms ordered K-fastest ((r/128)*ceil(K/64) + c/4);
+ *           inside an atom the byte of (r, c) is at (r%32)*16 + ((r%128)/32)*4
+ *           + c%4.  Pad bytes are written as 0.  Size: nvfp4_sf_bytes().
+ *   Y       bf16 (or fp32 with NVFP4_FLAG_F32_OUT), row-major [M, N], row
+ *           stride ldy elements (16-byte aligned rows).
+ *
+ * Shape limits: K % 64 == 0, N % 8 == 0, M >= 0 (M == 0 is a no-op),
+ * 1 <= nseg <= NVFP4_MAX_SEGMENTS, segment offsets strictly increasing from 0
+ * to N (each a multiple of 8).
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nvfp4_stream_t; /* same type as cudaStream_t */
+
+#define NVFP4_MAX_SEGMENTS 8
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad segment table, unknown flag */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 64, N % 8, too many segments, size overflow */
+    NVFP4_ERR_MISALIGNED = 3,         /* pointer or row stride not 16-byte aligned */
+    NVFP4_ERR_NONFINITE = 4,          /* device saw a non-finite amax or static scale */
+    NVFP4_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+    NVFP4_ERR_TIMEOUT = 6,            /* a bounded pipeline wait inside a kernel ran out */
+    NVFP4_ERR_WORKSPACE = 7,          /* workspace null or smaller than nvfp4_workspace_bytes() */
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 8  /* current device is not sm_100 */
+} nvfp4_status;
+
+/* Flags for nvfp4_gemm / nvfp4_linear / nvfp4_linear_fused. */
+#define NVFP4_FLAG_F32_OUT 0x1u              /* write fp32 instead of bf16 (numerics checks) */
+#define NVFP4_FLAG_COLLAPSED_MAX_SCALE 0x2u  /* negative control: every column uses s_x * max(s_w),
+                                                the mismatch of the paper's §6; never for serving */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *nvfp4_status_string(nvfp4_status st);
+
+/* Bytes of a physical SF buffer for `rows` rows of K elements:
+ * ceil(rows/128)*128 * ceil(K/16/4)*4.  Returns 0 for invalid input. */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k);
+
+/* Bytes of device workspace that nvfp4_quantize_act / nvfp4_linear /
+ * nvfp4_linear_fused / nvfp4_pack_weight need for an [m, k] activation
+ * (or weight) operand.  The workspace needs no initialisation and its contents
+ * after a call are unspecified; calls sharing one workspace must be ordered on
+ * one stream. */
+size_t nvfp4_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/* Activation quantization (step 1).
+ * x           device bf16 [m, k], row stride ldx.
+ * gscale_in   device float: static (calibrated) global scale s_x, or NULL for
+ *             the dynamic per-tensor scale s_x = amax(|x|) / 2688 computed on the GPU.
+ * gscale_out  device float, receives the s_x used (may alias gscale_in).
+ * q           device [m, k/2] bytes (packed codes).
+ * sf          device nvfp4_sf_bytes(m, k) bytes (swizzled block scales, pads zeroed).
+ * workspace   device, >= nvfp4_workspace_bytes(m, 0, k) bytes. */
+nvfp4_status nvfp4_quantize_act(const void *x, int64_t m, int64_t k, int64_t ldx,
+                                const float *gscale_in, float *gscale_out,
+                                uint8_t *q, uint8_t *sf,
+                                void *workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* Offline weight packing: the same codec applied to W [n, k] (row stride ldw),
+ * one global scale per segment (module) of rows.
+ * seg_offsets host int64[nseg+1] (0 = seg_offsets[0] < ... < seg_offsets[nseg] = n),
+ *             or NULL with nseg == 1 for a single module.
+ * gscale_in   device float[nseg] static scales, or NULL for amax/2688 per segment.
+ * gscale_out  device float[nseg], receives the scales used.
+ * q, sf       device outputs as for nvfp4_quantize_act, for n rows.
+ * workspace   device, >= nvfp4_workspace_bytes(n, 0, k) bytes. */
+nvfp4_status nvfp4_pack_weight(const void *w, int64_t n, int64_t k, int64_t ldw,
+                               const int64_t *seg_offsets, int nseg,
+                               const float *gscale_in, float *gscale_out,
+                               uint8_t *q, uint8_t *sf,
+                               void *workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* Block-scaled FP4 GEMM + epilogue on already-quantized operands (steps 2, 3).
+ * qx, sfx, s_x  device activation codes [m, k/2], scales, global scale (1 float).
+ * qw, sfw       device weight codes [n, k/2] and scales.
+ * seg_offsets   host int64[nseg+1] column segments (NULL with nseg == 1).
+ * seg_gscales   device float[nseg] weight global scale per segment.
+ * y             device [m, n] output (bf16, or fp32 with NVFP4_FLAG_F32_OUT), row stride ldy.
+ * flags         NVFP4_FLAG_* bits.
+ * Needs no workspace. */
+nvfp4_status nvfp4_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m,
+                        const uint8_t *qw, const uint8_t *sfw, int64_t n, int64_t k,
+                        const int64_t *seg_offsets, const float *seg_gscales, int nseg,
+                        void *y, int64_t ldy, unsigned flags, nvfp4_stream_t stream);
+
+/* The whole layer for one module: quantize x, GEMM against the packed weight,
+ * epilogue with s_x * s_w.  act_gscale: device static s_x or NULL (dynamic).
+ * workspace >= nvfp4_workspace_bytes(m, n, k). */
+nvfp4_status nvfp4_linear(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,
+                          const uint8_t *qw, const uint8_t *sfw, const float *w_gscale, int64_t n,
+                          void *y, int64_t ldy, unsigned flags,
+                          void *workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* The whole layer for modules fused along N (e.g. q/k/v/gate projections
+ * concatenated into one GEMM), each keeping its own weight global scale:
+ * column j of segment i is scaled by s_x * seg_gscales[i] (paper §6).
+ * seg_offsets host int64[nseg+1]; seg_gscales device float[nseg]. */
+nvfp4_status nvfp4_linear_fused(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,
+                                const uint8_t *qw, const uint8_t *sfw, int64_t n,
+                                const int64_t *seg_offsets, const float *seg_gscales, int nseg,
+                                void *y, int64_t ldy, unsigned flags,
+                                void *workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* Synchronizes `stream`, then returns and clears the current device's error
+ * word: NVFP4_ERR_NONFINITE, NVFP4_ERR_TIMEOUT, or NVFP4_OK. */
+nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream);
+
+/* Upper bound, in nanoseconds, of every pipeline wait inside the GEMM kernel
+ * on the current process (default 2e9).  A wait that runs out makes the kernel
+ * record NVFP4_ERR_TIMEOUT, drain its in-flight copies, release its tensor
+ * memory and return.  Values below 1000 are raised to 1000. */
+void nvfp4_set_wait_timeout_ns(uint64_t ns);
+
+/* Library version string. */
+const char *nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

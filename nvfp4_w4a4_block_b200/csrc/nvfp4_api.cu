@@ -1,0 +1,446 @@
+// nvfp4_api.cu -- the C ABI declared in include/nvfp4.h: host-side validation,
+// workspace layout, TMA descriptor construction and kernel launches.
+//
+// Workspace layout (caller-owned device memory, no initialisation needed):
+//   [0, 32 KB)            amax partials: up to 8 segments x 1024 CTAs x 4 bytes
+//   [32 KB, +m*k/2)       activation codes Qx (nvfp4_linear*)
+//   [.., +sf_bytes(m,k))  activation block scales SFx (nvfp4_linear*)
+//   +16 bytes             activation global scale s_x (nvfp4_linear*)
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/nvfp4.h"
+#include "gemm_sm100.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+using namespace nvfp4;
+
+constexpr size_t kPartialBytes = 32 * 1024;
+constexpr int kMaxPartials = 1024;
+constexpr size_t kAlign = 256;
+
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+struct DeviceInfo {
+    bool ready = false;
+    nvfp4_status status = NVFP4_OK;
+    int sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+// One-time per-device set-up: capability check, SM count, kernel attributes,
+// driver entry point for tensor-map encoding.
+nvfp4_status device_setup(int *sms)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return NVFP4_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, sm = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        if (major != 10 || minor != 0) {
+            d.ready = true;
+            d.status = NVFP4_ERR_UNSUPPORTED_DEVICE;
+            return d.status;
+        }
+        if (cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::SMEM_ALLOC) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        if (g_encode == nullptr) {
+            cudaDriverEntryPointQueryResult q;
+            void *fn = nullptr;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return NVFP4_ERR_CUDA;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        d.sms = sm;
+        d.status = NVFP4_OK;
+        d.ready = true;
+    }
+    *sms = d.sms;
+    return d.status;
+}
+
+// Shared argument checks for an operand [rows, k] in bf16 with row stride ld.
+nvfp4_status check_bf16_operand(const void *x, int64_t rows, int64_t k, int64_t ld)
+{
+    if (rows < 0 || k <= 0 || ld < k)
+        return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t(1) << 31) || k > (int64_t(1) << 30))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > 0 && x == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x) || (ld * 2) % 16 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+// Validates a segment table over `total` rows/columns and copies its ends.
+nvfp4_status read_segments(const int64_t *offsets, int nseg, int64_t total, int64_t *ends)
+{
+    if (nseg < 1 || nseg > NVFP4_MAX_SEGMENTS)
+        return nseg > NVFP4_MAX_SEGMENTS ? NVFP4_ERR_UNSUPPORTED_SHAPE : NVFP4_ERR_INVALID_ARG;
+    if (offsets == nullptr) {
+        if (nseg != 1)
+            return NVFP4_ERR_INVALID_ARG;
+        ends[0] = total;
+        return NVFP4_OK;
+    }
+    if (offsets[0] != 0 || offsets[nseg] != total)
+        return NVFP4_ERR_INVALID_ARG;
+    for (int i = 0; i < nseg; ++i)
+        if (offsets[i + 1] <= offsets[i])
+            return NVFP4_ERR_INVALID_ARG;
+    for (int i = 0; i < nseg; ++i) {
+        if (offsets[i + 1] % 8 != 0)
+            return NVFP4_ERR_UNSUPPORTED_SHAPE;
+        ends[i] = offsets[i + 1];
+    }
+    return NVFP4_OK;
+}
+
+int amax_grid(int sms, int64_t rows, int64_t k)
+{
+    const int64_t units = rows * (k / 8);
+    int64_t g = (units + kQuantThreads * 4 - 1) / (kQuantThreads * 4);
+    if (g > 4 * sms)
+        g = 4 * sms;
+    if (g > kMaxPartials)
+        g = kMaxPartials;
+    return static_cast<int>(g < 1 ? 1 : g);
+}
+
+int quant_grid(int sms, int64_t rows, int64_t k)
+{
+    const int64_t units = rows * (k / 8) + (int64_t(128) * (k / 64));   // + pad words
+    int64_t g = (units + kQuantThreads - 1) / kQuantThreads;
+    if (g > 8 * sms)
+        g = 8 * sms;
+    return static_cast<int>(g < 1 ? 1 : g);
+}
+
+// amax partials (dynamic mode) + encode, rows split into segments.
+nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx, const int64_t *seg_ends, int nseg,
+                             const float *static_scale, float *scale_out, uint8_t *q, uint8_t *sf,
+                             uint32_t *partials, int sms, cudaStream_t stream)
+{
+    const int ga = amax_grid(sms, rows, k);
+    if (static_scale == nullptr) {
+        int64_t begin = 0;
+        for (int s = 0; s < nseg; ++s) {
+            AmaxParams ap;
+            ap.x = static_cast<const uint16_t *>(x);
+            ap.row_begin = begin;
+            ap.row_end = seg_ends[s];
+            ap.k = k;
+            ap.ldx = ldx;
+            ap.partial = partials + s * ga;
+            amax_partial_kernel<<<ga, kQuantThreads, 0, stream>>>(ap);
+            begin = seg_ends[s];
+        }
+    }
+    QuantParams qp;
+    memset(&qp, 0, sizeof qp);
+    qp.x = static_cast<const uint16_t *>(x);
+    qp.rows = rows;
+    qp.k = k;
+    qp.ldx = ldx;
+    qp.q = reinterpret_cast<uint32_t *>(q);
+    qp.sf = sf;
+    qp.rows_pad = (rows + 127) / 128 * 128;
+    qp.kb_pad = ((k / 16) + 3) / 4 * 4;
+    qp.nseg = nseg;
+    for (int s = 0; s < nseg; ++s)
+        qp.seg_end[s] = seg_ends[s];
+    qp.static_scale = static_scale;
+    qp.partial = partials;
+    qp.npartial = ga;
+    qp.scale_out = scale_out;
+    quantize_kernel<<<quant_grid(sms, rows, k), kQuantThreads, 0, stream>>>(qp);
+    return cuda_status(cudaGetLastError());
+}
+
+nvfp4_status make_map(CUtensorMap *map, const void *base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows)
+{
+    cuuint64_t dims[2] = {inner_bytes, rows};
+    cuuint64_t strides[1] = {inner_bytes};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
+                         const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
+                         const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms,
+                         cudaStream_t stream)
+{
+    CUtensorMap ta, tb;
+    nvfp4_status st = make_map(&ta, qx, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(m), gemm::BM);
+    if (st != NVFP4_OK)
+        return st;
+    st = make_map(&tb, qw, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n), gemm::BN);
+    if (st != NVFP4_OK)
+        return st;
+    gemm::Params p;
+    memset(&p, 0, sizeof p);
+    p.sfa = sfx;
+    p.sfb = sfw;
+    p.m = static_cast<int>(m);
+    p.n = static_cast<int>(n);
+    p.k = static_cast<int>(k);
+    p.tiles_m = static_cast<int>((m + gemm::BM - 1) / gemm::BM);
+    p.tiles_n = static_cast<int>((n + gemm::BN - 1) / gemm::BN);
+    p.atoms_k = k / 64;
+    p.k_stages = static_cast<int>((k + gemm::BK - 1) / gemm::BK);
+    p.y = y;
+    p.ldy = ldy;
+    p.s_x = s_x;
+    p.s_w = seg_gscales;
+    p.nseg = nseg;
+    for (int s = 0; s < nseg; ++s)
+        p.seg_end[s] = static_cast<int>(seg_ends[s]);
+    p.flags = flags;
+    p.timeout_ns = g_timeout_ns.load();
+    const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    gemm::nvfp4_gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_ALLOC, stream>>>(ta, tb, p);
+    return cuda_status(cudaGetLastError());
+}
+
+struct WorkspaceLayout {
+    size_t q_off, sf_off, scale_off, total;
+};
+
+WorkspaceLayout workspace_layout(int64_t m, int64_t k)
+{
+    WorkspaceLayout w;
+    w.q_off = kPartialBytes;
+    w.sf_off = align_up(w.q_off + static_cast<size_t>(m) * static_cast<size_t>(k / 2), kAlign);
+    w.scale_off = align_up(w.sf_off + nvfp4_sf_bytes(m, k), kAlign);
+    w.total = w.scale_off + kAlign;
+    return w;
+}
+
+nvfp4_status check_gemm_args(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
+                             const uint8_t *sfw, int64_t n, int64_t k, const float *seg_gscales, const void *y,
+                             int64_t ldy, unsigned flags)
+{
+    if (m < 0 || n <= 0 || k <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (flags & ~(NVFP4_FLAG_F32_OUT | NVFP4_FLAG_COLLAPSED_MAX_SCALE))
+        return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0 || n % 8 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (m > (int64_t(1) << 31) - 256 || n > (int64_t(1) << 31) - 256 || k > (int64_t(1) << 30))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (qw == nullptr || sfw == nullptr || seg_gscales == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (m > 0 && (qx == nullptr || sfx == nullptr || s_x == nullptr || y == nullptr))
+        return NVFP4_ERR_INVALID_ARG;
+    if (ldy < n)
+        return NVFP4_ERR_INVALID_ARG;
+    const int64_t esz = (flags & NVFP4_FLAG_F32_OUT) ? 4 : 2;
+    if (!aligned16(qx) || !aligned16(sfx) || !aligned16(qw) || !aligned16(sfw) || !aligned16(y) ||
+        (ldy * esz) % 16 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *nvfp4_status_string(nvfp4_status st)
+{
+    switch (st) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case NVFP4_ERR_NONFINITE: return "non-finite global scale";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_TIMEOUT: return "pipeline wait timed out";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
+    }
+    return "unknown status";
+}
+
+const char *nvfp4_version(void) { return "nvfp4-b200 0.1"; }
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k)
+{
+    if (rows < 0 || k <= 0 || k % 16 != 0)
+        return 0;
+    const size_t rows_pad = static_cast<size_t>((rows + 127) / 128 * 128);
+    const size_t cols_pad = static_cast<size_t>(((k / 16) + 3) / 4 * 4);
+    return rows_pad * cols_pad;
+}
+
+size_t nvfp4_workspace_bytes(int64_t m, int64_t n, int64_t k)
+{
+    (void)n;
+    if (m < 0 || k <= 0 || k % 16 != 0)
+        return 0;
+    return workspace_layout(m, k).total;
+}
+
+void nvfp4_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns < 1000 ? 1000 : ns); }
+
+nvfp4_status nvfp4_quantize_act(const void *x, int64_t m, int64_t k, int64_t ldx, const float *gscale_in,
+                                float *gscale_out, uint8_t *q, uint8_t *sf, void *workspace, size_t ws_bytes,
+                                nvfp4_stream_t stream)
+{
+    nvfp4_status st = check_bf16_operand(x, m, k, ldx);
+    if (st != NVFP4_OK)
+        return st;
+    if (gscale_out == nullptr || (m > 0 && (q == nullptr || sf == nullptr)))
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(sf))
+        return NVFP4_ERR_MISALIGNED;
+    if (gscale_in == nullptr && (workspace == nullptr || ws_bytes < kPartialBytes))
+        return NVFP4_ERR_WORKSPACE;
+    if (m == 0)
+        return NVFP4_OK;
+    int sms = 0;
+    if ((st = device_setup(&sms)) != NVFP4_OK)
+        return st;
+    int64_t end = m;
+    return launch_quantize(x, m, k, ldx, &end, 1, gscale_in, gscale_out, q, sf, static_cast<uint32_t *>(workspace),
+                           sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_pack_weight(const void *w, int64_t n, int64_t k, int64_t ldw, const int64_t *seg_offsets,
+                               int nseg, const float *gscale_in, float *gscale_out, uint8_t *q, uint8_t *sf,
+                               void *workspace, size_t ws_bytes, nvfp4_stream_t stream)
+{
+    nvfp4_status st = check_bf16_operand(w, n, k, ldw);
+    if (st != NVFP4_OK)
+        return st;
+    if (n <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    int64_t ends[NVFP4_MAX_SEGMENTS];
+    if ((st = read_segments(seg_offsets, nseg, n, ends)) != NVFP4_OK)
+        return st;
+    if (gscale_out == nullptr || q == nullptr || sf == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(sf))
+        return NVFP4_ERR_MISALIGNED;
+    if (gscale_in == nullptr && (workspace == nullptr || ws_bytes < kPartialBytes))
+        return NVFP4_ERR_WORKSPACE;
+    int sms = 0;
+    if ((st = device_setup(&sms)) != NVFP4_OK)
+        return st;
+    return launch_quantize(w, n, k, ldw, ends, nseg, gscale_in, gscale_out, q, sf,
+                           static_cast<uint32_t *>(workspace), sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
+                        const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_offsets,
+                        const float *seg_gscales, int nseg, void *y, int64_t ldy, unsigned flags,
+                        nvfp4_stream_t stream)
+{
+    nvfp4_status st = check_gemm_args(qx, sfx, s_x, m, qw, sfw, n, k, seg_gscales, y, ldy, flags);
+    if (st != NVFP4_OK)
+        return st;
+    int64_t ends[NVFP4_MAX_SEGMENTS];
+    if ((st = read_segments(seg_offsets, nseg, n, ends)) != NVFP4_OK)
+        return st;
+    if (m == 0)
+        return NVFP4_OK;
+    int sms = 0;
+    if ((st = device_setup(&sms)) != NVFP4_OK)
+        return st;
+    return launch_gemm(qx, sfx, s_x, m, qw, sfw, n, k, ends, nseg, seg_gscales, y, ldy, flags, sms,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_linear_fused(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,
+                                const uint8_t *qw, const uint8_t *sfw, int64_t n, const int64_t *seg_offsets,
+                                const float *seg_gscales, int nseg, void *y, int64_t ldy, unsigned flags,
+                                void *workspace, size_t ws_bytes, nvfp4_stream_t stream)
+{
+    nvfp4_status st = check_bf16_operand(x, m, k, ldx);
+    if (st != NVFP4_OK)
+        return st;
+    const WorkspaceLayout wl = workspace_layout(m, k);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    // The GEMM's activation operands come from the workspace (the scale slot
+    // stands in for s_x: a NULL act_gscale selects the dynamic scale).
+    st = check_gemm_args(ws + wl.q_off, ws + wl.sf_off, reinterpret_cast<const float *>(ws + wl.scale_off), m, qw,
+                         sfw, n, k, seg_gscales, y, ldy, flags);
+    if (st != NVFP4_OK)
+        return st;
+    int64_t ends[NVFP4_MAX_SEGMENTS];
+    if ((st = read_segments(seg_offsets, nseg, n, ends)) != NVFP4_OK)
+        return st;
+    if (m == 0)
+        return NVFP4_OK;
+    if (workspace == nullptr || ws_bytes < wl.total || !aligned16(workspace))
+        return NVFP4_ERR_WORKSPACE;
+    int sms = 0;
+    if ((st = device_setup(&sms)) != NVFP4_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float *sx = reinterpret_cast<float *>(ws + wl.scale_off);
+    int64_t end = m;
+    st = launch_quantize(x, m, k, ldx, &end, 1, act_gscale, sx, ws + wl.q_off, ws + wl.sf_off,
+                         reinterpret_cast<uint32_t *>(ws), sms, s);
+    if (st != NVFP4_OK)
+        return st;
+    return launch_gemm(ws + wl.q_off, ws + wl.sf_off, sx, m, qw, sfw, n, k, ends, nseg, seg_gscales, y, ldy, flags,
+                       sms, s);
+}
+
+nvfp4_status nvfp4_linear(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,
+                          const uint8_t *qw, const uint8_t *sfw, const float *w_gscale, int64_t n, void *y,
+                          int64_t ldy, unsigned flags, void *workspace, size_t ws_bytes, nvfp4_stream_t stream)
+{
+    return nvfp4_linear_fused(x, m, k, ldx, act_gscale, qw, sfw, n, nullptr, w_gscale, 1, y, ldy, flags, workspace,
+                              ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream)
+{
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, nvfp4::g_device_error, sizeof v) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(nvfp4::g_device_error, &zero, sizeof zero) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+    }
+    return static_cast<nvfp4_status>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,299 @@
+// quantize.cuh -- NVFP4 quantization kernels (activations per call, weights offline).
+//
+// Method ("Why Gated DeltaNet Survives 4-Bit Quantization", §2 "NVFP4"): each run
+// of 16 consecutive elements along K gets one E4M3 block scale set to blockmax/6
+// relative to an FP32 per-tensor global scale; elements are rounded to E2M1.
+// Arithmetic order (identical on the CPU reference, element for element):
+//   s    = amax / 2688                        (fp32, dynamic mode; else the given s)
+//   sb   = E4M3_rn_satfinite(min(bmax / (s*6), 448))   (0 when s*6 == 0)
+//   d    = value(sb) * s;  r = d == 0 ? 0 : min(1/d, FLT_MAX)
+//   code = E2M1_rn_satfinite(x * r)           two codes per byte, lower K index low
+//
+// Kernel design (HBM-bound): one thread owns 8 consecutive bf16 (one 16-byte
+// load), two neighbouring lanes own a 16-element block and exchange their
+// halves' maxima with one shuffle; eight lanes cover four blocks of one row,
+// whose four scale bytes are contiguous in the tensor-core layout and leave in
+// one 32-bit store.  The codes of a thread leave in one 32-bit store, so a warp
+// writes 128 contiguous bytes.  The amax pass reduces in bf16 bit space
+// (|x| bits = x & 0x7FFF; integer max orders finite < inf < NaN) and writes one
+// partial per CTA, which the encode pass reduces again -- no atomics, no
+// workspace initialisation, deterministic.
+#pragma once
+
+#include <cfloat>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace nvfp4 {
+
+constexpr int kQuantThreads = 256;
+constexpr int kMaxSeg = 8;
+
+__device__ __forceinline__ void raise_device_error(unsigned code)
+{
+    atomicCAS(&g_device_error, 0u, code);
+}
+
+// ------------------------------------------------------------------ helpers
+
+// |bf16| bit patterns: per-halfword unsigned max over a 16-byte chunk.
+__device__ __forceinline__ uint32_t absmax_bits8(const uint4 &v)
+{
+    const uint32_t m = 0x7FFF7FFFu;
+    uint32_t a = __vmaxu2(v.x & m, v.y & m);
+    uint32_t b = __vmaxu2(v.z & m, v.w & m);
+    uint32_t c = __vmaxu2(a, b);
+    return max(c >> 16, c & 0xFFFFu);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// E4M3 (satfinite, round-to-nearest-even) of a non-negative finite fp32 <= 448.
+__device__ __forceinline__ uint32_t f32_to_e4m3(float v)
+{
+    uint16_t h;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(v));
+    return h & 0xFFu;
+}
+
+// Exact decode of an E4M3 byte (sign ignored: block scales are non-negative).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code)
+{
+    uint32_t h2;
+    uint16_t in = static_cast<uint16_t>(code & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// Eight fp32 -> four bytes of E2M1 codes (round-to-nearest-even, saturating);
+// element 2i in bits 8i..8i+3, element 2i+1 in bits 8i+4..8i+7.  The cvt puts its
+// first source operand in the high nibble, so each pair is passed (odd, even).
+__device__ __forceinline__ uint32_t f32x8_to_e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5,
+                                                    float v6, float v7)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return out;
+}
+
+__device__ __forceinline__ int64_t sf_atom_offset(int64_t row, int64_t kb, int64_t kb_pad)
+{
+    return ((row >> 7) * (kb_pad >> 2) + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+}
+
+// ------------------------------------------------------------------ amax
+
+struct AmaxParams {
+    const uint16_t *x;
+    int64_t row_begin, row_end, k, ldx;
+    uint32_t *partial;   // one entry per CTA
+};
+
+__global__ void __launch_bounds__(kQuantThreads) amax_partial_kernel(AmaxParams p)
+{
+    const int64_t upr = p.k >> 3;                          // 16-byte units per row
+    const int64_t rows = p.row_end - p.row_begin;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    // Each thread walks four interleaved streams of units; (row, col) advance
+    // by a precomputed step so that no division sits in the loop.
+    const int64_t step = 4 * nthreads, step_r = step / upr, step_c = step % upr;
+    int64_t row[4], col[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t u = gtid + j * nthreads;
+        row[j] = u / upr;
+        col[j] = u % upr;
+    }
+    uint32_t best = 0;
+    while (row[0] < rows) {
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (row[j] < rows)
+                v[j] = __ldg(reinterpret_cast<const uint4 *>(p.x + (p.row_begin + row[j]) * p.ldx + col[j] * 8));
+            else
+                v[j] = make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            best = max(best, absmax_bits8(v[j]));
+            col[j] += step_c;
+            row[j] += step_r;
+            if (col[j] >= upr) {
+                col[j] -= upr;
+                ++row[j];
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        best = max(best, __shfl_xor_sync(0xFFFFFFFFu, best, o));
+    __shared__ uint32_t warp_best[kQuantThreads / 32];
+    if ((threadIdx.x & 31) == 0)
+        warp_best[threadIdx.x >> 5] = best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < kQuantThreads / 32; ++w)
+            b = max(b, warp_best[w]);
+        p.partial[blockIdx.x] = b;
+    }
+}
+
+// ------------------------------------------------------------------ encode
+
+struct QuantParams {
+    const uint16_t *x;
+    int64_t rows, k, ldx;
+    uint32_t *q;                 // packed codes, viewed as 32-bit words (8 codes)
+    uint8_t *sf;                 // physical scale buffer
+    int64_t rows_pad, kb_pad;    // padded scale-layout extents
+    int nseg;
+    int64_t seg_end[kMaxSeg];    // row end of each segment (last == rows)
+    const float *static_scale;   // [nseg] or nullptr (dynamic)
+    const uint32_t *partial;     // [nseg][npartial] amax partials (dynamic)
+    int npartial;
+    float *scale_out;            // [nseg]
+};
+
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
+{
+    __shared__ float s_scale[kMaxSeg];
+    __shared__ float s_dg[kMaxSeg];
+    const int lane = threadIdx.x & 31;
+
+    // Per-segment global scale: given, or amax / 2688 from the amax partials.
+    if (threadIdx.x < 32 * p.nseg && (threadIdx.x >> 5) < kMaxSeg) {
+        const int seg = threadIdx.x >> 5;
+        float s;
+        bool finite;
+        if (p.static_scale != nullptr) {
+            s = p.static_scale[seg];
+            finite = isfinite(s) && s >= 0.0f;
+        } else {
+            uint32_t b = 0;
+            for (int i = lane; i < p.npartial; i += 32)
+                b = max(b, p.partial[seg * p.npartial + i]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+            finite = b < 0x7F80u;
+            const float amax = __uint_as_float(b << 16);
+            s = __fdiv_rn(amax, 2688.0f);
+        }
+        if (lane == 0) {
+            if (!finite) {
+                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
+                s = 0.0f;
+            }
+            s_scale[seg] = s;
+            s_dg[seg] = __fmul_rn(s, 6.0f);
+            if (blockIdx.x == 0)
+                p.scale_out[seg] = s;
+        }
+    }
+    __syncthreads();
+
+    const int64_t upr = p.k >> 3;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    // Four interleaved unit streams per thread; (row, col) advance by a fixed
+    // step, so the loop holds no division.  Lane pairs (2i, 2i+1) always hold
+    // the two halves of one 16-element block, lanes 8g..8g+7 four aligned blocks
+    // of one row (nthreads is a multiple of 256 and upr of 8).
+    const int64_t step = 4 * nthreads, step_r = step / upr, step_c = step % upr;
+    int64_t row[4], col[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t u = gtid + j * nthreads;
+        row[j] = u / upr;
+        col[j] = u % upr;
+    }
+    // Warp-uniform trip count: lane 0's first stream decides.
+    int64_t wrow = __shfl_sync(0xFFFFFFFFu, row[0], 0);
+    int64_t wcol = __shfl_sync(0xFFFFFFFFu, col[0], 0);
+
+    while (wrow < p.rows) {
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (row[j] < p.rows)
+                v[j] = __ldg(reinterpret_cast<const uint4 *>(p.x + row[j] * p.ldx + col[j] * 8));
+            else
+                v[j] = make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const bool active = row[j] < p.rows;
+            const int64_t r_ = active ? row[j] : 0;
+            const int64_t c8 = col[j];
+
+            uint32_t bm = absmax_bits8(v[j]);
+            bm = max(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
+            const float bmax = __uint_as_float(bm << 16);
+
+            int seg = 0;
+#pragma unroll
+            for (int s = 0; s < kMaxSeg - 1; ++s)
+                seg += (s + 1 < p.nseg && r_ >= p.seg_end[s]) ? 1 : 0;
+            const float s = s_scale[seg];
+            const float dg = s_dg[seg];
+
+            const float sbf = (dg == 0.0f) ? 0.0f : fminf(__fdiv_rn(bmax, dg), 448.0f);
+            const uint32_t sb = f32_to_e4m3(sbf);
+            const float d = __fmul_rn(e4m3_to_f32(sb), s);
+            const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX);
+
+            const uint32_t w0 = v[j].x, w1 = v[j].y, w2 = v[j].z, w3 = v[j].w;
+            const uint32_t codes = f32x8_to_e2m1x8(
+                __fmul_rn(bf16lo(w0), r), __fmul_rn(bf16hi(w0), r), __fmul_rn(bf16lo(w1), r),
+                __fmul_rn(bf16hi(w1), r), __fmul_rn(bf16lo(w2), r), __fmul_rn(bf16hi(w2), r),
+                __fmul_rn(bf16lo(w3), r), __fmul_rn(bf16hi(w3), r));
+            if (active)
+                p.q[r_ * upr + c8] = codes;
+
+            // Lanes 8g, 8g+2, 8g+4, 8g+6 hold the scales of four consecutive blocks
+            // (k-block index = c8/2, aligned to 4) of one row: one 32-bit store.
+            const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
+            const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
+            const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sb, 6);
+            if (active && (lane & 7) == 0)
+                *reinterpret_cast<uint32_t *>(p.sf + sf_atom_offset(r_, c8 >> 1, p.kb_pad)) =
+                    sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+
+            col[j] += step_c;
+            row[j] += step_r;
+            if (col[j] >= upr) {
+                col[j] -= upr;
+                ++row[j];
+            }
+        }
+        wcol += step_c;
+        wrow += step_r;
+        if (wcol >= upr) {
+            wcol -= upr;
+            ++wrow;
+        }
+    }
+
+    // Zero the scale bytes of the pad rows [rows, rows_pad): 4 bytes per (row, atom).
+    const int64_t pad_words = (p.rows_pad - p.rows) * (p.kb_pad >> 2);
+    for (int64_t i = gtid; i < pad_words; i += nthreads) {
+        const int64_t row = p.rows + i / (p.kb_pad >> 2);
+        const int64_t kb = (i % (p.kb_pad >> 2)) << 2;
+        *reinterpret_cast<uint32_t *>(p.sf + sf_atom_offset(row, kb, p.kb_pad)) = 0u;
+    }
+}
+
+}  // namespace nvfp4

@@ -197,12 +197,17 @@ def linear_reference(x_bits: np.ndarray, w_bits: np.ndarray, seg_offsets: Sequen
     """The whole layer on the CPU: dynamic (or given) activation scale, per-segment
     weight scales, quantize both operands, fp64 GEMM on the selected rows.
 
-    Returns dict(y=fp64 [len(rows), N], s_x, s_w, qx, sfx, qw, sfw)."""
+    Returns dict(y=fp64 [len(rows), N], s_x, s_w, qx, sfx, qw, sfw); with `rows`
+    given, qx/sfx hold only those rows."""
     s_x = global_scale(amax(x_bits)) if act_scale is None else np.float32(act_scale)
     s_w = segment_scales(w_bits, seg_offsets) if w_scales is None else np.asarray(w_scales, np.float32)
-    qx, sfx = quantize(x_bits, s_x)
     qw, sfw = quantize(w_bits, row_scales_from_segments(seg_offsets, s_w))
     if rows is None:
-        rows = np.arange(x_bits.shape[0])
-    y = linear_rows(qx, sfx, s_x, rows, qw, sfw, col_scales(seg_offsets, s_w))
+        qx, sfx = quantize(x_bits, s_x)
+        sel = np.arange(x_bits.shape[0])
+    else:
+        # Only the selected rows are quantized; the global scale above is the whole tensor's.
+        qx, sfx = quantize(np.ascontiguousarray(x_bits[np.asarray(rows)]), s_x)
+        sel = np.arange(len(rows))
+    y = linear_rows(qx, sfx, s_x, sel, qw, sfw, col_scales(seg_offsets, s_w))
     return dict(y=y, s_x=s_x, s_w=s_w, qx=qx, sfx=sfx, qw=qw, sfw=sfw)

@@ -1,0 +1,125 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry point
+include/nvfp4.h declares, and rejects bad arguments on the host before any CUDA
+call.  (No compute call is made here.)"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_w4a4_block_b200 as nv
+from nvfp4_w4a4_block_b200 import build as nvbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    nvbuild.build()
+    return nv.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(L, name), name
+    assert set(names) == set(nv.EXPORTED)
+
+
+def test_status_strings(L):
+    for st in range(9):
+        assert nv.status_string(st) not in ("", "unknown status")
+    assert nv.status_string(99) == "unknown status"
+
+
+def test_sf_bytes_layout_sizes(L):
+    assert nv.sf_bytes(1, 64) == 128 * 4
+    assert nv.sf_bytes(128, 256) == 128 * 16
+    assert nv.sf_bytes(129, 320) == 256 * 20
+    assert nv.sf_bytes(16, 256) == 128 * 16
+    assert nv.sf_bytes(-1, 64) == 0 and nv.sf_bytes(4, 8) == 0
+
+
+def test_workspace_grows_with_activation(L):
+    a, b = nv.workspace_bytes(1, 0, 5120), nv.workspace_bytes(32, 0, 5120)
+    assert 0 < a < b
+    assert nv.workspace_bytes(8192, 17408, 5120) >= 8192 * 5120 // 2 + nv.sf_bytes(8192, 5120)
+
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: validation fails first
+MIS = 0x10001
+
+
+def test_quantize_validation(L):
+    f = L.nvfp4_quantize_act
+    assert f(None, 4, 64, 64, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, 4, 48, 48, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert f(MIS, 4, 64, 64, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_MISALIGNED
+    assert f(FAKE, 4, 64, 68, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_MISALIGNED
+    assert f(FAKE, 4, 64, 32, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, 4, 64, 64, None, None, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, 4, 64, 64, None, FAKE, FAKE, FAKE, None, 0, None) == nv.ERR_WORKSPACE
+    assert f(FAKE, -1, 64, 64, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, 0, 64, 64, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.OK     # empty: no-op
+
+
+def _segs(*v):
+    return (ctypes.c_int64 * len(v))(*v)
+
+
+def test_gemm_validation(L):
+    g = L.nvfp4_gemm
+    ok = dict(qx=FAKE, sfx=FAKE, sx=FAKE, m=4, qw=FAKE, sfw=FAKE, n=64, k=128, seg=None, sw=FAKE, nseg=1, y=FAKE,
+              ldy=64, flags=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["qx"], a["sfx"], a["sx"], a["m"], a["qw"], a["sfw"], a["n"], a["k"], a["seg"], a["sw"], a["nseg"],
+                 a["y"], a["ldy"], a["flags"], None)
+
+    assert call(k=96) == nv.ERR_UNSUPPORTED_SHAPE
+    assert call(n=60, ldy=60) == nv.ERR_UNSUPPORTED_SHAPE
+    assert call(qw=None) == nv.ERR_INVALID_ARG
+    assert call(sw=None) == nv.ERR_INVALID_ARG
+    assert call(y=MIS) == nv.ERR_MISALIGNED
+    assert call(ldy=60) == nv.ERR_INVALID_ARG
+    assert call(ldy=68) == nv.ERR_MISALIGNED
+    assert call(flags=0x8) == nv.ERR_INVALID_ARG
+    assert call(nseg=2) == nv.ERR_INVALID_ARG                       # NULL table needs nseg == 1
+    assert call(seg=_segs(0, 32, 64), nseg=2, m=0) == nv.OK
+    assert call(seg=_segs(0, 32, 60), nseg=2) == nv.ERR_INVALID_ARG  # last != N
+    assert call(seg=_segs(0, 36, 64), nseg=2) == nv.ERR_UNSUPPORTED_SHAPE
+    assert call(seg=_segs(0, 32, 32, 64), nseg=3) == nv.ERR_INVALID_ARG
+    assert call(seg=_segs(*range(0, 80, 8)), nseg=9, n=72, ldy=72) == nv.ERR_UNSUPPORTED_SHAPE
+    assert call(m=0) == nv.OK
+
+
+def test_linear_validation(L):
+    f = L.nvfp4_linear
+    assert f(FAKE, 4, 128, 128, None, FAKE, FAKE, FAKE, 64, FAKE, 64, 0, None, 0, None) == nv.ERR_WORKSPACE
+    assert f(FAKE, 4, 128, 128, None, FAKE, FAKE, FAKE, 64, FAKE, 64, 0, FAKE, 16, None) == nv.ERR_WORKSPACE
+    assert f(None, 4, 128, 128, None, FAKE, FAKE, FAKE, 64, FAKE, 64, 0, FAKE, 1 << 30, None) == nv.ERR_INVALID_ARG
+
+
+def test_pack_validation(L):
+    f = L.nvfp4_pack_weight
+    assert f(FAKE, 64, 128, 128, _segs(0, 16, 64), 2, None, FAKE, FAKE, FAKE, None, 0, None) == nv.ERR_WORKSPACE
+    assert f(FAKE, 64, 128, 128, _segs(0, 70, 64), 2, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == \
+        nv.ERR_INVALID_ARG
+    assert f(FAKE, 0, 128, 128, None, 1, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import importlib
+    mod = importlib.import_module("nvfp4_w4a4_block_b200")
+    monkeypatch.setattr(mod, "_lib", None)
+    monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        mod.lib()

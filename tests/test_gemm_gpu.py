@@ -1,0 +1,191 @@
+"""GPU parity of the block-scaled FP4 GEMM and of the whole linear layer
+against the CPU oracle (fp64 GEMM on the identical dequantized operands).
+
+The operands the GPU quantized are first asserted bit-exact with the oracle's,
+so any GEMM error is the kernel's.  Tolerance (tests/_helpers.py): fp32
+output within 1e-3 of max(|R|, row RMS); bf16 output additionally within its
+own rounding (2^-8 relative), and equal to the RNE rounding of the same
+kernel's fp32 output.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from nvfp4_w4a4_block_b200 import workloads as W
+
+from _helpers import assert_gemm_close, bf16_rne_from_f32, to_cuda_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import nvfp4_w4a4_block_b200 as nv
+    nv.lib()
+    return nv
+
+
+def _bf16_to_f64(t):
+    import torch
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _layer(nv, xb, wb, seg_offsets, rows=None, act_static=None, flags=0):
+    """Run the whole layer on the GPU; return (y_gpu [rows], oracle dict)."""
+    import torch
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), seg_offsets)
+    g = None if act_static is None else torch.tensor([act_static], dtype=torch.float32, device="cuda")
+    y = nv.linear_fused(x, pw, act_gscale=g, flags=flags)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    ref = oracle.linear_reference(xb, wb, seg_offsets, rows=rows, act_scale=act_static)
+    assert pw.gscale.cpu().numpy().tobytes() == ref["s_w"].tobytes()
+    if rows is None:
+        yg = y
+    else:
+        yg = y[torch.as_tensor(np.asarray(rows), device="cuda")]
+    return yg, ref, pw
+
+
+@pytest.mark.parametrize("m,n,k,segs", [
+    (16, 128, 256, None),          # tiny workload shape
+    (1, 8, 64, None),              # smallest: one row, one column group, one K atom
+    (3, 96, 64, None),
+    (128, 256, 256, None),         # exactly one tile, one stage
+    (300, 600, 1088, None),        # ragged M, N and K-stage tails, several tiles
+    (257, 520, 320, [0, 256, 520]),
+    (64, 1040, 2048, [0, 512, 768, 1024, 1040]),
+    (130, 264, 5120, [0, 136, 264]),
+])
+def test_gemm_parity_random(nv, m, n, k, segs):
+    import torch
+    seg_rows = None if segs is None else [segs[i + 1] - segs[i] for i in range(len(segs) - 1)]
+    xb, wb, off = W.random_case(7, m, n, k, seg_rows=seg_rows)
+    y32, ref, pw = _layer(nv, xb, wb, off, flags=nv.FLAG_F32_OUT)
+    assert_gemm_close(y32.cpu().numpy(), ref["y"], bf16=False)
+    ybf = nv.linear_fused(to_cuda_bf16(xb), pw)
+    torch.cuda.synchronize()
+    assert_gemm_close(_bf16_to_f64(ybf), ref["y"], bf16=True)
+    # the bf16 output is exactly the RNE rounding of the fp32 result
+    assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), bf16_rne_from_f32(y32.cpu().numpy()))
+
+
+def test_gemm_exact_on_representable_operands(nv):
+    """E2M1 grid values x power-of-two block magnitudes under power-of-two global
+    scales quantize losslessly, so the layer must reproduce X.W^T (fp64 via
+    NumPy) to fp32 accumulation accuracy."""
+    import torch
+    rng = np.random.default_rng(12)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -.5, -1, -1.5, -2, -3, -4, -6])
+    m, n, k = 200, 264, 512
+
+    def rep(rows):
+        v = rng.choice(grid, size=(rows, k))
+        v[:, ::16] = 6.0
+        return v * np.repeat(2.0 ** rng.integers(-3, 3, size=(rows, k // 16)), 16, axis=1)
+
+    x, w = rep(m), rep(n)
+    xb, wb = W.f32_to_bf16_bits(x), W.f32_to_bf16_bits(w)
+    pw = nv.pack_weight(to_cuda_bf16(wb), gscale=torch.tensor([2.0 ** -5], device="cuda"))
+    y = nv.linear(to_cuda_bf16(xb), pw, act_gscale=torch.tensor([2.0 ** -6], device="cuda"),
+                  flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+    exact = x @ w.T
+    err = np.abs(y.cpu().numpy().astype(np.float64) - exact)
+    assert (err <= 1e-6 * np.maximum(np.abs(exact), 1.0)).all()
+
+
+def test_fused_segments_match_separate_modules_and_collapsed_mode_fails(nv):
+    """Per-segment epilogue == separate per-module GEMMs; the collapsed-max mode
+    (the serving mismatch of the paper's §6) mis-scales the smaller-scale module
+    by the scale ratio."""
+    import torch
+    m, k = 96, 512
+    xb, wb, off = W.random_case(9, m, 512, k, seg_rows=[256, 256])
+    wf = W.bf16_bits_to_f32(wb).copy()
+    wf[256:] *= 2.75 / 2.0                          # segment scales differ ~2.75x
+    wb = W.f32_to_bf16_bits(wf)
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    fused = nv.linear_fused(x, pw, flags=nv.FLAG_F32_OUT)
+    for i in range(2):
+        pwi = nv.pack_weight(to_cuda_bf16(np.ascontiguousarray(wb[off[i]:off[i + 1]])))
+        yi = nv.linear(x, pwi, flags=nv.FLAG_F32_OUT)
+        torch.cuda.synchronize()
+        assert torch.equal(yi, fused[:, off[i]:off[i + 1]])
+    bad = nv.linear_fused(x, pw, flags=nv.FLAG_F32_OUT | nv.FLAG_COLLAPSED_MAX_SCALE)
+    torch.cuda.synchronize()
+    s_w = pw.gscale.cpu().numpy()
+    ratio = s_w.max() / s_w.min()
+    assert ratio > 2.5
+    small = int(np.argmin(s_w))
+    sl = slice(off[small], off[small + 1])
+    e = (torch.linalg.norm(bad[:, sl] - fused[:, sl]) / torch.linalg.norm(fused[:, sl])).item()
+    assert abs(e - (ratio - 1)) < 1e-3
+    ref = oracle.linear_reference(xb, wb, off)
+    assert_gemm_close(fused.cpu().numpy(), ref["y"], bf16=False)
+
+
+def test_gemm_entry_on_prequantized_operands(nv):
+    import torch
+    xb, wb, off = W.random_case(10, 200, 384, 768)
+    x = to_cuda_bf16(xb)
+    qx, sfx, sx = nv.quantize_act(x)
+    pw = nv.pack_weight(to_cuda_bf16(wb))
+    y = nv.gemm(qx, sfx, sx, 200, pw, flags=nv.FLAG_F32_OUT)
+    y2 = nv.linear(x, pw, flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+
+
+def test_static_activation_scale(nv):
+    xb, wb, off = W.random_case(11, 140, 256, 640)
+    y, ref, _ = _layer(nv, xb, wb, off, act_static=0.004, flags=nv.FLAG_F32_OUT)
+    assert_gemm_close(y.cpu().numpy(), ref["y"], bf16=False)
+
+
+def test_zero_rows_is_a_noop(nv):
+    import torch
+    pw = nv.pack_weight(to_cuda_bf16(W.random_case(0, 1, 64, 128)[1]))
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    y = nv.linear(x, pw)
+    assert y.shape == (0, 64)
+
+
+# ----------------------------------------------------------------- workloads
+
+def _rows_sample(m, seed, n_rand):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([np.arange(min(m, 64)), rng.integers(0, m, n_rand),
+                                     np.arange(max(0, m - 32), m)]))
+
+
+def test_tiny_workload_full(nv):
+    wl = W.TINY
+    y, ref, _ = _layer(nv, wl.x(), wl.w(), wl.seg_offsets)
+    assert_gemm_close(_bf16_to_f64(y), ref["y"], bf16=True)
+
+
+@pytest.mark.parametrize("m", W.DECODE_M)
+def test_decode_workload_full(nv, m):
+    wl = W.DECODE
+    y, ref, _ = _layer(nv, wl.x(m), wl.w(), wl.seg_offsets)
+    assert_gemm_close(_bf16_to_f64(y), ref["y"], bf16=True)
+
+
+@pytest.mark.parametrize("wl", [W.PREFILL, W.FUSED_QKVG], ids=lambda w: w.name)
+def test_prefill_workloads_sampled_rows(nv, wl):
+    rows = _rows_sample(wl.m, wl.cfg_id, 64)
+    y, ref, _ = _layer(nv, wl.x(), wl.w(), wl.seg_offsets, rows=rows)
+    assert_gemm_close(_bf16_to_f64(y), ref["y"], bf16=True)
+
+
+def test_long_prefill_workload_sampled_rows(nv):
+    wl = W.LONG_DOWN
+    rows = _rows_sample(wl.m, wl.cfg_id, 32)[::2]
+    y, ref, _ = _layer(nv, wl.x(), wl.w(), wl.seg_offsets, rows=rows)
+    assert_gemm_close(_bf16_to_f64(y), ref["y"], bf16=True)

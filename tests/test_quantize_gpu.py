@@ -1,0 +1,173 @@
+"""GPU parity of the NVFP4 quantization kernels against the CPU oracle.
+
+Codes, scale bytes (physical tensor-core layout, pads included) and the global
+scale must match bit for bit; both sides take every rounding decision in fp32
+with the same operation order.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from nvfp4_w4a4_block_b200 import workloads as W
+
+from _helpers import to_cuda_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import nvfp4_w4a4_block_b200 as nv
+    nv.lib()
+    return nv
+
+
+def _run_quant(nv, bits, static=None):
+    import torch
+    x = to_cuda_bf16(bits)
+    g = None if static is None else torch.tensor([static], dtype=torch.float32, device="cuda")
+    q, sf, s = nv.quantize_act(x, gscale=g)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    return q.cpu().numpy(), sf.cpu().numpy(), np.float32(s.item())
+
+
+def _expect(bits, static=None):
+    s = oracle.global_scale(oracle.amax(bits)) if static is None else np.float32(static)
+    q, sf = oracle.quantize(bits, s)
+    return q, oracle.sf_to_physical(sf, bits.shape[1]), s
+
+
+def _compare(nv, bits, static=None):
+    qg, sfg, sg = _run_quant(nv, bits, static)
+    qo, sfo, so = _expect(bits, static)
+    assert sg.tobytes() == np.float32(so).tobytes()
+    assert sfg.shape == sfo.shape
+    if not np.array_equal(sfg, sfo):
+        bad = np.flatnonzero(sfg != sfo)
+        raise AssertionError(f"{bad.size} scale bytes differ, first at {bad[0]}: gpu {sfg[bad[0]]:#x} "
+                             f"oracle {sfo[bad[0]]:#x}")
+    if not np.array_equal(qg, qo):
+        bad = np.argwhere(qg != qo)
+        r, c = bad[0]
+        raise AssertionError(f"{len(bad)} code bytes differ, first at {r},{c}: gpu {qg[r, c]:#x} "
+                             f"oracle {qo[r, c]:#x}")
+
+
+@pytest.mark.parametrize("m,k", [(1, 64), (2, 128), (16, 256), (127, 320), (300, 1088), (129, 5120),
+                                 (37, 17408), (1000, 64)])
+def test_quantize_random_shapes_dynamic(nv, m, k):
+    x, _, _ = W.random_case(3, m, 8, k)
+    _compare(nv, x)
+
+
+@pytest.mark.parametrize("static", [2.0 ** -9, 1e-3, 0.37, 1e-6, 0.0])
+def test_quantize_static_scale(nv, static):
+    x, _, _ = W.random_case(4, 200, 8, 512)
+    _compare(nv, x, static)
+
+
+def test_quantize_every_bf16_value_on_identity_scale(nv):
+    """Global scale 2^-8 and a 6.0 in every block make the element divisor exactly
+    1, so each bf16 value in [-6, 6] is encoded as itself: every tie, every
+    sub-grid value, both zeros."""
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = W.bf16_bits_to_f32(bits)
+    keep = bits[np.isfinite(vals) & (np.abs(vals) <= 6.0)]
+    per_block = 15
+    nblk = (keep.size + per_block - 1) // per_block
+    pad = nblk * per_block - keep.size
+    body = np.concatenate([keep, np.zeros(pad, np.uint16)]).reshape(nblk, per_block)
+    six = W.f32_to_bf16_bits(np.full((nblk, 1), 6.0, np.float32))
+    blocks = np.concatenate([six, body], axis=1)                      # [nblk, 16]
+    k = 1024
+    rows = (nblk * 16 + k - 1) // k
+    flat = np.concatenate([blocks.reshape(-1), np.tile(six.reshape(-1)[:1], rows * k - nblk * 16)])
+    _compare(nv, flat.reshape(rows, k), 2.0 ** -8)
+
+
+def test_quantize_ties_under_power_of_two_block_scales(nv):
+    """Exact ties (0.25, 0.75, ... 5 times the divisor) at many block magnitudes."""
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    rows = []
+    for j in range(-10, 6):
+        blk = np.concatenate([[6.0], ties, -ties, [0.0]]).astype(np.float32) * np.float32(2.0 ** j)
+        rows.append(np.tile(blk, 4))
+    x = W.f32_to_bf16_bits(np.stack(rows))
+    _compare(nv, x, 2.0 ** -8)
+    _compare(nv, x)
+
+
+def test_quantize_zero_and_negative_zero(nv):
+    x = np.zeros((3, 64), np.uint16)
+    x[1, ::2] = 0x8000                                  # -0.0
+    _compare(nv, x)
+    _compare(nv, x, 0.5)
+
+
+def test_quantize_strided_rows(nv):
+    import torch
+    xb, _, _ = W.random_case(5, 64, 8, 256)
+    big = np.zeros((64, 384), np.uint16)
+    big[:, :256] = xb
+    xt = to_cuda_bf16(big)[:, :256]
+    q, sf, s = nv.quantize_act(xt)
+    torch.cuda.synchronize()
+    qo, sfo, so = _expect(xb)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(sf.cpu().numpy(), sfo)
+
+
+def test_quantize_nonfinite_sets_device_error(nv):
+    import torch
+    x = np.zeros((4, 64), np.uint16)
+    x[2, 5] = 0x7F80                                     # +inf
+    xt = to_cuda_bf16(x)
+    nv.quantize_act(xt)
+    assert nv.get_device_error() == nv.ERR_NONFINITE
+    assert nv.get_device_error() == nv.OK               # cleared
+    nv.quantize_act(to_cuda_bf16(np.ones((4, 64), np.uint16)))
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+
+
+@pytest.mark.parametrize("wl", [W.TINY, W.DECODE, W.PREFILL, W.FUSED_QKVG], ids=lambda w: w.name)
+def test_quantize_workload_activations(nv, wl):
+    _compare(nv, wl.x())
+
+
+def test_quantize_long_prefill_activations_sampled_rows(nv):
+    """32768 x 17408 (the standalone-quantize workload): the global scale comes
+    from the whole tensor; codes and scales are compared on sampled rows."""
+    import torch
+    wl = W.LONG_DOWN
+    xb = wl.x()
+    x = to_cuda_bf16(xb)
+    q, sf, s = nv.quantize_act(x)
+    torch.cuda.synchronize()
+    s_ref = oracle.global_scale(oracle.amax(xb))
+    assert np.float32(s.item()).tobytes() == s_ref.tobytes()
+    rows = np.unique(np.concatenate([np.arange(0, 128), np.random.default_rng(0).integers(0, wl.m, 128),
+                                     np.arange(wl.m - 64, wl.m)]))
+    qo, sfo = oracle.quantize(np.ascontiguousarray(xb[rows]), s_ref)
+    qg = q[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    assert np.array_equal(qg, qo)
+    sf_h = sf.cpu().numpy()
+    offs = np.array([[oracle.sf_offset(int(r), c, wl.k) for c in range(wl.k // 16)] for r in rows])
+    assert np.array_equal(sf_h[offs], sfo)
+
+
+@pytest.mark.parametrize("wl", [W.DECODE, W.FUSED_QKVG], ids=lambda w: w.name)
+def test_pack_weight_per_segment_scales(nv, wl):
+    import torch
+    wb = wl.w()
+    pw = nv.pack_weight(to_cuda_bf16(wb), wl.seg_offsets)
+    torch.cuda.synchronize()
+    s_ref = oracle.segment_scales(wb, wl.seg_offsets)
+    assert pw.gscale.cpu().numpy().tobytes() == s_ref.tobytes()
+    qo, sfo = oracle.quantize(wb, oracle.row_scales_from_segments(wl.seg_offsets, s_ref))
+    assert np.array_equal(pw.q.cpu().numpy(), qo)
+    assert np.array_equal(pw.sf.cpu().numpy(), oracle.sf_to_physical(sfo, wl.k))
