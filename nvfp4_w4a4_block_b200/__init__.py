@@ -218,8 +218,8 @@ def gemm(qx, sfx, s_x, m: int, pw: PackedWeight, out=None, flags: int = 0, strea
     """Block-scaled FP4 GEMM + per-segment global-scale epilogue on quantized operands."""
     y = _out(m, pw.n, pw.q.device, flags, out)
     arr, nseg = _seg_array(pw.seg_offsets)
-    st = lib().nvfp4_gemm(_ptr(qx), _ptr(sfx), _ptr(s_x), m, _ptr(pw.q), _ptr(pw.sf), pw.n, pw.k, arr, nseg,
-                          _ptr(pw.gscale), _ptr(y), y.stride(0), flags, _stream(stream))
+    st = lib().nvfp4_gemm(_ptr(qx), _ptr(sfx), _ptr(s_x), m, _ptr(pw.q), _ptr(pw.sf), pw.n, pw.k, arr,
+                          _ptr(pw.gscale), nseg, _ptr(y), y.stride(0), flags, _stream(stream))
     _check(st, "nvfp4_gemm")
     return y
 
@@ -234,7 +234,7 @@ def linear_fused(x, pw: PackedWeight, act_gscale=None, out=None, flags: int = 0,
     ws = workspace(m, pw.n, k, x.device) if ws is None else ws
     arr, nseg = _seg_array(pw.seg_offsets)
     st = lib().nvfp4_linear_fused(_ptr(x), m, k, x.stride(0), _ptr(act_gscale), _ptr(pw.q), _ptr(pw.sf), pw.n, arr,
-                                  nseg, _ptr(pw.gscale), _ptr(y), y.stride(0), flags, _ptr(ws), ws.numel(),
+                                  _ptr(pw.gscale), nseg, _ptr(y), y.stride(0), flags, _ptr(ws), ws.numel(),
                                   _stream(stream))
     _check(st, "nvfp4_linear_fused")
     return y
