@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 W4A4 linear layer on B200.
+
+Primary line (the decode-shaped workload): one step = the fused gate+up layer
+(K=5120, N=34816 as two modules with their own weight global scales) called
+once each for M = 1, 8 and 32 tokens, the whole path per call (dynamic
+activation amax, quantize, block-scaled FP4 GEMM, per-segment epilogue, bf16
+out).  value = algorithmic HBM bytes of the step / device time (GB/s).  Every
+call reads a different copy of the packed weights (copies rotate over >= 4x
+the 126 MB L2), so each call streams its weights from HBM.
+
+The same JSON line carries the dominant kernel's roofline (the GEMM, timed
+alone with CUDA events on its stream), the end-to-end number through host
+buffers, the clocks seen during the timed region, the CPU oracle as a
+baseline, and the other workloads (prefill TFLOP/s, standalone quantize GB/s)
+under "workloads".
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nvfp4|reference]
+Under torchrun each rank runs its own replica of the step on its own GPU
+(independent batches, no data-path collective: weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 linear TFLOP/s (prefill) & GB/s (decode, quantize) as % of B200 roofline"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP4_OVER_BF16 = 4.0          # nominal dense ratio 9 PFLOP/s fp4 : 2.25 PFLOP/s bf16
+
+
+# ----------------------------------------------------------------------------- peaks / clocks
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=FALLBACK_BF16_TFLOPS,
+                    bf16_tflops_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 50 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def _target(self):
+        import torch
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            return vis.split(",")[self.dev] if vis else str(self.dev)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self._target(), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.reader.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def dev_bf16_from_bits(bits):
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def gen_device(shape, dist, seed, outlier_frac=0.0, outlier_mult=1.0, sigma=1.0):
+    """Seeded synthetic bf16 tensor generated on the GPU (Philox), with the
+    workloads' distributions: N(0, sigma) or Student-t nu=3, plus scaled
+    outlier channels."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    if dist == "normal":
+        x = torch.randn(shape, generator=g, device="cuda", dtype=torch.float32) * sigma
+    else:  # Student-t, nu = 3: z / sqrt(chi2_3 / 3)
+        z = torch.randn(shape, generator=g, device="cuda", dtype=torch.float32)
+        c = torch.zeros(shape, device="cuda", dtype=torch.float32)
+        for _ in range(3):
+            c.add_(torch.randn(shape, generator=g, device="cuda", dtype=torch.float32).square_())
+        x = z / torch.sqrt(c / 3.0)
+        del z, c
+    if outlier_frac > 0:
+        k = shape[1]
+        n_out = max(1, int(round(outlier_frac * k)))
+        cols = torch.randperm(k, generator=g, device="cuda")[:n_out]
+        x[:, cols] *= outlier_mult
+    return x.to(torch.bfloat16)
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def time_reps(fn, reps, warmup, flush=None):
+    """Per-rep CUDA-event times (ms) on the current stream, L2 flushed before each rep."""
+    import torch
+    for _ in range(warmup):
+        if flush is not None:
+            flush()
+        fn()
+    torch.cuda.synchronize()
+    out = []
+    s = torch.cuda.current_stream()
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        fn()
+        e1.record(s)
+        out.append((e0, e1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in out]
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nvfp4_w4a4_block_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+        e = d[kernel][workload]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- workload bytes
+
+def decode_call_bytes(m, n, k, dynamic=True, gemm_only=False):
+    """Algorithmic HBM bytes of one decode-shaped call: packed weights (codes
+    N*K/2 + scales N*K/16), activations in (bf16, read twice in dynamic mode:
+    amax and encode), activation codes+scales written and read back
+    (0.5625 B/elem each way), bf16 output."""
+    w = n * k // 2 + n * k // 16
+    act_q = m * k // 2 + m * k // 16
+    y = 2 * m * n
+    if gemm_only:
+        return w + act_q + y
+    x = 2 * m * k * (2 if dynamic else 1)
+    return w + x + 2 * act_q + y
+
+
+# ----------------------------------------------------------------------------- nvfp4 arm
+
+def run_nvfp4(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import nvfp4_w4a4_block_b200 as nv
+    from nvfp4_w4a4_block_b200 import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    nv.lib()
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    wl = W.DECODE
+    n, k, off = wl.n, wl.k, wl.seg_offsets
+    ms = list(W.DECODE_M)
+    mmax = max(ms)
+
+    # Packed weights: one pack, replicated into enough copies to defeat the L2.
+    w = gen_device((n, k), "normal", 1000 + rank, sigma=0.02)
+    w[off[1]:] *= 2.75                                       # second module: distinct global scale
+    pw0 = nv.pack_weight(w, off)
+    del w
+    wbytes = pw0.q.numel() + pw0.sf.numel()
+    copies = max(4, int(np.ceil(4 * L2_BYTES / wbytes)))
+    pws = [pw0] + [nv.PackedWeight(pw0.q.clone(), pw0.sf.clone(), pw0.gscale.clone(), pw0.n, pw0.k, pw0.seg_offsets)
+                   for _ in range(copies - 1)]
+    x_full = gen_device((mmax, k), "normal", 2000 + rank, wl.outlier_frac, wl.outlier_mult)
+    xs = {m: x_full[:m].contiguous() for m in ms}
+    ys = {m: torch.empty((m, n), dtype=torch.bfloat16, device="cuda") for m in ms}
+    wss = {m: torch.empty(nv.workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda") for m in ms}
+    torch.cuda.synchronize()
+
+    ctr = [0]
+
+    def step():
+        for m in ms:
+            pw = pws[ctr[0] % copies]
+            ctr[0] += 1
+            nv.linear_fused(xs[m], pw, out=ys[m], ws=wss[m])
+
+    step_bytes = sum(decode_call_bytes(m, n, k) for m in ms)
+    launches_per_step = 3 * len(ms)                          # amax, quantize, gemm per call
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if nv.get_device_error() != nv.OK:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- timed region: exactly K steps
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.15)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        step()
+    e1.record(s)
+    # The same step keeps running (untimed) for >= 0.6 s so that the clock
+    # sampler sees the load even when the timed region is short.
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < 0.6:
+        for _ in range(50):
+            step()
+        torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if clocks is not None:
+        clocks["window"] = "timed region + 0.6 s continuation of the same step"
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = e0.elapsed_time(e1)
+    if nv.get_device_error() != nv.OK:
+        raise RuntimeError("device error in the timed region")
+    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * step_bytes * args.steps / (ms_max * 1e-3) / 1e9
+
+    # ---- dominant kernel: the GEMM alone, per M (events on its stream)
+    per_m = {}
+    for m in ms:
+        qx, sfx, sx = nv.quantize_act(xs[m])
+        ym = ys[m]
+        cnt = [0]
+
+        def g():
+            pw = pws[cnt[0] % copies]
+            cnt[0] += 1
+            nv.gemm(qx, sfx, sx, m, pw, out=ym)
+
+        def full():
+            pw = pws[cnt[0] % copies]
+            cnt[0] += 1
+            nv.linear_fused(xs[m], pw, out=ym, ws=wss[m])
+
+        tg = time_reps(g, 30, 5)
+        tf = time_reps(full, 30, 5)
+        gb = decode_call_bytes(m, n, k, gemm_only=True)
+        fb = decode_call_bytes(m, n, k)
+        per_m[str(m)] = dict(gemm_us=statistics.median(tg) * 1e3, gemm_gbs=gb / (statistics.median(tg) * 1e-3) / 1e9,
+                             call_us=statistics.median(tf) * 1e3, call_gbs=fb / (statistics.median(tf) * 1e-3) / 1e9,
+                             gemm_bytes=gb, call_bytes=fb)
+    gm = per_m[str(mmax)]
+    roofline = dict(bound="hbm", kernel="nvfp4_gemm_kernel", workload=f"decode M={mmax}",
+                    achieved=round(gm["gemm_gbs"], 1), peak=peaks["hbm_gbs"], unit="GB/s",
+                    frac=round(gm["gemm_gbs"] / peaks["hbm_gbs"], 4),
+                    traffic=committed_traffic("nvfp4_gemm_kernel", f"decode_M{mmax}"),
+                    algorithmic_bytes_per_launch=gm["gemm_bytes"], peak_source=peaks["source"])
+
+    # ---- end to end through host buffers (pinned), H2D of X and D2H of Y inside the region
+    hx = {m: xs[m].cpu().pin_memory() for m in ms}
+    hy = {m: torch.empty((m, n), dtype=torch.bfloat16).pin_memory() for m in ms}
+    dx = {m: torch.empty_like(xs[m]) for m in ms}
+
+    def e2e_step():
+        for m in ms:
+            pw = pws[ctr[0] % copies]
+            ctr[0] += 1
+            dx[m].copy_(hx[m], non_blocking=True)
+            nv.linear_fused(dx[m], pw, out=ys[m], ws=wss[m])
+            hy[m].copy_(ys[m], non_blocking=True)
+
+    te = time_reps(e2e_step, max(10, min(args.steps, 200)), 3)
+    e2e_ms = statistics.median(te)
+    h2d = sum(xs[m].numel() * 2 for m in ms)
+    d2h = sum(m * n * 2 for m in ms)
+    e2e = dict(value=round(step_bytes / (e2e_ms * 1e-3) / 1e9, 1), unit="GB/s", h2d_bytes_per_step=h2d,
+               d2h_bytes_per_step=d2h, ms_per_step=round(e2e_ms, 4))
+
+    del pws, pw0
+    torch.cuda.empty_cache()
+    workloads = {}
+    if rank == 0 and not args.skip_secondary:
+        workloads = secondary_workloads(nv, W, peaks, fp4_peak)
+        workloads["decode_per_m"] = per_m
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3 block16, fp32 accumulate, bf16 out)",
+        "data": "synthetic (seeded Philox on device: X ~ N(0,1) with 0.5% outlier channels x50, "
+                "W ~ N(0,0.02) / N(0,0.055) per module)",
+        "config": {"workload": "decode-shaped fused gate+up: M in {1,8,32} tokens (one call each per step), "
+                               "K=5120, N=34816 = 2 x 17408 modules with distinct weight global scales, "
+                               "dynamic activation scale",
+                   "l2": f"inputs larger than L2: packed weights rotate over {copies} copies "
+                         f"({copies * wbytes / 2**20:.0f} MiB), a different copy per call",
+                   "parallelism": f"replicas x{world} (one independent step per GPU)"},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp4_tflops": round(fp4_peak, 1),
+                  "fp4_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} "
+                                f"(nominal dense fp4:bf16 ratio)"},
+        "workloads": workloads,
+    }
+    return line
+
+
+def secondary_workloads(nv, W, peaks, fp4_peak):
+    """Prefill-shaped GEMMs (TFLOP/s vs the dense FP4 peak) and the standalone
+    quantize (GB/s vs HBM), each rep timed alone with the L2 flushed before it."""
+    import torch
+    out = {}
+    flush_buf = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device="cuda")
+
+    def flush():
+        flush_l2(flush_buf)
+
+    for wl in (W.PREFILL, W.FUSED_QKVG, W.LONG_DOWN):
+        m, n, k, off = wl.m, wl.n, wl.k, wl.seg_offsets
+        sig = torch.tensor(wl.seg_sigma, dtype=torch.float32)
+        w = gen_device((n, k), "normal", 31 + wl.cfg_id)
+        for i in range(len(off) - 1):
+            w[off[i]:off[i + 1]] *= float(sig[i])
+        pw = nv.pack_weight(w, off)
+        x = gen_device((m, k), wl.x_dist, 41 + wl.cfg_id, wl.outlier_frac, wl.outlier_mult)
+        y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(nv.workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda")
+        qx, sfx, sx = nv.quantize_act(x)
+        reps = 10 if wl is not W.LONG_DOWN else 6
+        tf = statistics.median(time_reps(lambda: nv.linear_fused(x, pw, out=y, ws=ws), reps, 3, flush))
+        tg = statistics.median(time_reps(lambda: nv.gemm(qx, sfx, sx, m, pw, out=y), reps, 3, flush))
+        fl = 2.0 * m * n * k
+        wb = w.to(torch.bfloat16)
+        tb = statistics.median(time_reps(lambda: torch.matmul(x, wb.t()), reps, 2, flush))
+        out[wl.name] = dict(
+            call_ms=round(tf, 4), call_tflops=round(fl / (tf * 1e-3) / 1e12, 1),
+            gemm_ms=round(tg, 4), gemm_tflops=round(fl / (tg * 1e-3) / 1e12, 1),
+            gemm_frac_fp4_peak=round(fl / (tg * 1e-3) / 1e12 / fp4_peak, 4),
+            call_frac_fp4_peak=round(fl / (tf * 1e-3) / 1e12 / fp4_peak, 4),
+            bf16_matmul_ms=round(tb, 4), speedup_over_bf16_call=round(tb / tf, 3), segments=len(off) - 1)
+        del w, wb, pw, x, y, ws, qx, sfx
+        torch.cuda.empty_cache()
+
+    # standalone activation quantize on the long-prefill tensor (HBM-bound)
+    wl = W.LONG_DOWN
+    m, k = wl.m, wl.k
+    x = gen_device((m, k), "normal", 77, wl.outlier_frac, wl.outlier_mult)
+    q = torch.empty((m, k // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty(nv.sf_bytes(m, k), dtype=torch.uint8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    td = statistics.median(time_reps(lambda: nv.quantize_act(x, q=q, sf=sf, gscale_out=s), 10, 3, flush))
+    static = s.clone()
+    ts = statistics.median(time_reps(lambda: nv.quantize_act(x, gscale=static, q=q, sf=sf, gscale_out=s), 10, 3,
+                                     flush))
+    elems = m * k
+    b_static = elems * (2 + 0.5 + 1 / 16)
+    b_dyn = elems * (4 + 0.5 + 1 / 16)
+    out["quantize_32768x17408"] = dict(
+        dynamic_ms=round(td, 4), dynamic_gbs=round(b_dyn / (td * 1e-3) / 1e9, 1),
+        dynamic_frac_hbm=round(b_dyn / (td * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        static_ms=round(ts, 4), static_gbs=round(b_static / (ts * 1e-3) / 1e9, 1),
+        static_frac_hbm=round(b_static / (ts * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        bytes_dynamic=int(b_dyn), bytes_static=int(b_static))
+    del x, q, sf, flush_buf
+    torch.cuda.empty_cache()
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_step(sample_cols: int):
+    """One decode-shaped step on the CPU oracle over a column sample; returns
+    (seconds, algorithmic bytes of the sampled work, threads)."""
+    import numpy as np
+
+    import oracle
+    from nvfp4_w4a4_block_b200 import workloads as W
+    wl = W.DECODE
+    k = wl.k
+    rng = np.random.default_rng(5)
+    wb = W.f32_to_bf16_bits(rng.standard_normal((sample_cols, k), dtype=np.float32) * np.float32(0.02))
+    s_w = oracle.segment_scales(wb, [0, sample_cols])
+    qw, sfw = oracle.quantize(wb, s_w[0])                  # offline packing, not timed
+    x32 = wl.x(max(W.DECODE_M))
+    t0 = time.perf_counter()
+    for m in W.DECODE_M:
+        xb = np.ascontiguousarray(x32[:m])
+        s_x = oracle.global_scale(oracle.amax(xb))
+        qx, sfx = oracle.quantize(xb, s_x)
+        oracle.linear_rows(qx, sfx, s_x, np.arange(m), qw, sfw, np.full(sample_cols, s_w[0], np.float32))
+    dt = time.perf_counter() - t0
+    nbytes = sum(decode_call_bytes(m, sample_cols, k) for m in W.DECODE_M)
+    return dt, nbytes, oracle.num_threads()
+
+
+def cpu_baseline(sample_cols=8704):
+    dt, nbytes, threads = oracle_step(sample_cols)
+    return dict(value=round(nbytes / dt / 1e9, 4), unit="GB/s", cores=threads, kind="oracle",
+                sample=f"one decode step (M=1,8,32; K=5120) over {sample_cols} of 34816 weight columns, "
+                       f"fp64 GEMM, {dt:.1f} s")
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on this machine's host cores.
+    Each step is the decode step over a column sample sized so that the whole
+    --warmup + --steps run takes about 90 s."""
+    if rank != 0:
+        return None
+    t_cal, _, _ = oracle_step(512)
+    per_col = t_cal / 512
+    budget = min(0.5, 90.0 / (args.steps + args.warmup))
+    cols = int(max(64, min(34816, round(budget / per_col / 8) * 8)))
+    for _ in range(args.warmup):
+        oracle_step(cols)
+    times, nbytes, threads = [], 0, 1
+    for _ in range(args.steps):
+        dt, nbytes, threads = oracle_step(cols)
+        times.append(dt)
+    total = sum(times)
+    value = nbytes * args.steps / total / 1e9
+    sample = f"one decode step (M=1,8,32; K=5120) over {cols} of 34816 weight columns per step"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle GEMM)",
+        "data": "synthetic (seeded NumPy PCG64)",
+        "config": {"workload": "decode-shaped fused gate+up, M in {1,8,32}, K=5120, N=34816 (column sample)",
+                   "parallelism": "host cores of rank 0"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="nvfp4", choices=["nvfp4", "reference"])
+    ap.add_argument("--skip-secondary", action="store_true", help="primary line only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import datetime
+
+    import torch
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_nvfp4(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
