@@ -478,11 +478,18 @@ def oracle_step(sample_cols: int):
     return dt, nbytes, oracle.num_threads()
 
 
-def cpu_baseline(sample_cols=8704):
-    dt, nbytes, threads = oracle_step(sample_cols)
-    return dict(value=round(nbytes / dt / 1e9, 4), unit="GB/s", cores=threads, kind="oracle",
-                sample=f"one decode step (M=1,8,32; K=5120) over {sample_cols} of 34816 weight columns, "
-                       f"fp64 GEMM, {dt:.1f} s")
+def cpu_baseline(target_s=10.0):
+    """The oracle on the full decode step (all 34816 columns), repeated until
+    about target_s seconds of CPU work."""
+    total_t, total_b, reps, threads = 0.0, 0, 0, 1
+    while total_t < target_s and reps < 50:
+        dt, nbytes, threads = oracle_step(34816)
+        total_t += dt
+        total_b += nbytes
+        reps += 1
+    return dict(value=round(total_b / total_t / 1e9, 4), unit="GB/s", cores=threads, kind="oracle",
+                sample=f"{reps} x one full decode step (M=1,8,32; K=5120; N=34816; weights pre-packed), "
+                       f"fp64 GEMM, {total_t:.1f} s")
 
 
 def run_reference(args, rank, world):
@@ -517,6 +524,79 @@ def run_reference(args, rank, world):
     }
 
 
+
+# ----------------------------------------------------------------------------- profiling cases
+
+def _prof_gemm(m, n, k, seg_offsets, launches, dist="normal"):
+    import torch
+
+    import nvfp4_w4a4_block_b200 as nv
+    w = gen_device((n, k), "normal", 5, sigma=0.02)
+    pw = nv.pack_weight(w, seg_offsets)
+    del w
+    x = gen_device((m, k), dist, 6, 0.005, 50.0)
+    qx, sfx, sx = nv.quantize_act(x)
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(launches):
+        nv.gemm(qx, sfx, sx, m, pw, out=y)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+
+
+def _prof_quantize(m, k, launches, static):
+    import torch
+
+    import nvfp4_w4a4_block_b200 as nv
+    x = gen_device((m, k), "normal", 7, 0.005, 50.0)
+    q = torch.empty((m, k // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty(nv.sf_bytes(m, k), dtype=torch.uint8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    nv.quantize_act(x, q=q, sf=sf, gscale_out=s)
+    g = s.clone() if static else None
+    torch.cuda.synchronize()
+    for _ in range(launches):
+        nv.quantize_act(x, gscale=g, q=q, sf=sf, gscale_out=s)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+
+
+def _prof_decode_call(m, launches):
+    import torch
+
+    import nvfp4_w4a4_block_b200 as nv
+    n, k, off = 34816, 5120, [0, 17408, 34816]
+    w = gen_device((n, k), "normal", 5, sigma=0.02)
+    pw = nv.pack_weight(w, off)
+    del w
+    x = gen_device((m, k), "normal", 6, 0.005, 50.0)
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(launches):
+        nv.linear_fused(x, pw, out=y)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+
+
+PROFILE_CASES = {
+    "gemm_decode_m32": lambda L: _prof_gemm(32, 34816, 5120, [0, 17408, 34816], L),
+    "gemm_prefill_8192x17408x5120": lambda L: _prof_gemm(8192, 17408, 5120, [0, 17408], L, "student_t3"),
+    "gemm_long_32768x5120x17408": lambda L: _prof_gemm(32768, 5120, 17408, [0, 5120], L),
+    "quantize_32768x17408_static": lambda L: _prof_quantize(32768, 17408, L, True),
+    "quantize_32768x17408_dynamic": lambda L: _prof_quantize(32768, 17408, L, False),
+    "decode_call_m32": lambda L: _prof_decode_call(32, L),
+}
+
+
+def run_profile_case(name, launches):
+    import torch
+
+    import nvfp4_w4a4_block_b200 as nv
+    torch.cuda.set_device(0)
+    nv.lib()
+    PROFILE_CASES[name](launches)
+    print(json.dumps({"profile_case": name, "launches": launches, "ok": True}))
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -527,6 +607,9 @@ def main():
     ap.add_argument("--impl", default="nvfp4", choices=["nvfp4", "reference"])
     ap.add_argument("--skip-secondary", action="store_true", help="primary line only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None, choices=sorted(PROFILE_CASES),
+                    help="run one kernel case a few times and exit (for ncu captures)")
+    ap.add_argument("--launches", type=int, default=3, help="launches of --profile-case")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -534,6 +617,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.profile_case is not None:
+        run_profile_case(args.profile_case, args.launches)
+        return
 
     if args.impl == "reference":
         line = run_reference(args, rank, world)
