@@ -1,0 +1,276 @@
+// gemm_decode.cuh -- block-scaled FP4 GEMM for few tokens (M <= 64), sm_100a.
+//
+// Same product and epilogue as gemm_sm100.cuh ("Why Gated DeltaNet Survives 4-Bit
+// Quantization", §2 "NVFP4"; per-module global scales of §6), organised for the
+// decode regime, which that paper calls weight-bandwidth-bound (§4) and where it
+// attributes the remaining loss to small-batch activation quantization (§9):
+//
+//   * Operands are swapped: the weight tile (128 rows of N) is the MMA's A operand,
+//     so it fills the 128 tensor-memory lanes, and the tokens are the MMA's N
+//     (T = 8, 16, 32 or 64).  No tile carries zero padding of the token dimension
+//     beyond T, and a stage is ~22-28 KB instead of 54 KB.
+//   * One CTA owns one 128-row weight tile over the whole K; two CTAs fit on an SM,
+//     so N/128 tiles (272 for N = 34816) are all resident at once and each SM keeps
+//     2 x (STAGES-1) weight stages in flight.
+//   * The kernel is launched with programmatic stream serialization: the producer
+//     streams the first STAGES weight stages before griddepcontrol.wait, i.e. while
+//     the activation quantizer that precedes it is still running, then loads the
+//     activation stages.
+//
+// Roles: warp 0 producer (TMA + bulk copies), warp 1 MMA issuer (one thread),
+// warps 2..5 epilogue (tcgen05.ld of the 128 x T accumulator, x alpha(n), bf16
+// stores of Y[t, n] -- 32 consecutive n per warp per token).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace nvfp4 {
+namespace decode {
+
+constexpr int BW = 128;                 // weight rows per tile (MMA M, TMEM lanes)
+constexpr int BK = 256;                 // K elements per stage (128 bytes per row)
+constexpr int KB = BK / 64;             // MMAs per stage
+constexpr int A_BYTES = BW * BK / 2;    // 16 KB of weight codes
+constexpr int SF_BYTES = KB * 512;      // one 128-row scale atom per K=64 block
+constexpr int THREADS = 192;
+constexpr uint64_t DRAIN_TIMEOUT_NS = 1000000000ull;
+constexpr int SMEM_LIMIT = 113 * 1024;  // two CTAs per SM
+
+constexpr unsigned FLAG_F32_OUT = 1u;
+constexpr unsigned FLAG_COLLAPSED = 2u;
+
+template <int T>
+struct Cfg {
+    static constexpr int B_BYTES = T * BK / 2;                              // token codes per stage
+    static constexpr int STAGE = A_BYTES + B_BYTES + 2 * SF_BYTES;
+    static constexpr int STAGES = (SMEM_LIMIT - 1024 - 256) / STAGE;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SF_BYTES;
+    static constexpr int OFF_BAR = OFF_SFB + STAGES * SF_BYTES;
+    static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 2) * 8;
+    static constexpr int SMEM_ALLOC = OFF_MISC + 64 + 1024;
+    static constexpr int TMEM_SFA = T;                 // columns after the accumulator
+    static constexpr int TMEM_SFB = T + KB * 4;
+    static constexpr int TMEM_COLS = (T + KB * 8 <= 32) ? 32 : (T + KB * 8 <= 64) ? 64 : 128;
+    static_assert(STAGES >= 3, "pipeline depth");
+    static_assert(SMEM_ALLOC <= SMEM_LIMIT, "two CTAs per SM");
+    static_assert(B_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+};
+
+struct Params {
+    const uint8_t *sfw;          // weight scales (A operand)
+    const uint8_t *sfx;          // activation scales (B operand), one 128-row block
+    int m, n, k;
+    int64_t atoms_k;             // K/64
+    int k_stages;
+    void *y;
+    int64_t ldy;
+    const float *s_x;
+    const float *s_w;
+    int nseg;
+    int seg_end[8];
+    unsigned flags;
+    uint64_t timeout_ns;
+};
+
+template <int T>
+__global__ void __launch_bounds__(THREADS, 2)
+    nvfp4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                             const Params p)
+{
+    using C = Cfg<T>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *acc_full = full + 2 * C::STAGES;
+    uint64_t *final_bar = acc_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int w0 = blockIdx.x * BW;              // first weight row (output column) of the tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(final_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tm_w);
+        prefetch_tensormap(&tm_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const int pre = min(C::STAGES, p.k_stages);
+            // Weight stages first: they do not depend on the preceding kernel.
+            for (int ks = 0; ks < pre; ++ks) {
+                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+                mbar_arrive_expect_tx(&full[ks], A_BYTES + C::B_BYTES + 2 * nkb * 512);
+                tma_load_2d(smem + C::OFF_A + ks * A_BYTES, &tm_w, ks * (BK / 2), w0, &full[ks]);
+                bulk_load(smem + C::OFF_SFA + ks * SF_BYTES,
+                          p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512, nkb * 512,
+                          &full[ks]);
+            }
+            pdl_wait_prerequisites();            // activation codes/scales are now written
+            for (int ks = 0; ks < pre; ++ks) {
+                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+                tma_load_2d(smem + C::OFF_B + ks * C::B_BYTES, &tm_x, ks * (BK / 2), 0, &full[ks]);
+                bulk_load(smem + C::OFF_SFB + ks * SF_BYTES, p.sfx + static_cast<int64_t>(ks * KB) * 512,
+                          nkb * 512, &full[ks]);
+            }
+            int stage = pre % C::STAGES;
+            uint32_t phase = (pre == C::STAGES) ? 1u : 0u;
+            int issued = pre;
+            for (int ks = pre; ks < p.k_stages; ++ks) {
+                if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns))
+                    break;
+                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+                mbar_arrive_expect_tx(&full[stage], A_BYTES + C::B_BYTES + 2 * nkb * 512);
+                tma_load_2d(smem + C::OFF_A + stage * A_BYTES, &tm_w, ks * (BK / 2), w0, &full[stage]);
+                bulk_load(smem + C::OFF_SFA + stage * SF_BYTES,
+                          p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512, nkb * 512,
+                          &full[stage]);
+                tma_load_2d(smem + C::OFF_B + stage * C::B_BYTES, &tm_x, ks * (BK / 2), 0, &full[stage]);
+                bulk_load(smem + C::OFF_SFB + stage * SF_BYTES, p.sfx + static_cast<int64_t>(ks * KB) * 512,
+                          nkb * 512, &full[stage]);
+                issued = ks + 1;
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            // Every stage issued must have landed before the CTA exits: the last
+            // min(STAGES, issued) issues are the only ones possibly in flight.
+            for (int j = 0; j < min(C::STAGES, issued); ++j) {
+                const int ks = issued - 1 - j;
+                const int s = ks % C::STAGES;
+                const uint32_t ph = static_cast<uint32_t>((ks / C::STAGES) & 1);
+                volatile int no_abort = 0;
+                if (!mbar_wait_bounded(&full[s], ph, &no_abort, DRAIN_TIMEOUT_NS))
+                    *abort_flag = 1;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc_nvfp4(BW, T);
+            const uint32_t sfa_t = tmem_base + C::TMEM_SFA;
+            const uint32_t sfb_t = tmem_base + C::TMEM_SFB;
+            const uint32_t a0 = smem_u32(smem + C::OFF_A), b0 = smem_u32(smem + C::OFF_B);
+            const uint32_t sfa0 = smem_u32(smem + C::OFF_SFA), sfb0 = smem_u32(smem + C::OFF_SFB);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int ks = 0; ks < p.k_stages; ++ks) {
+                if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    tc_cp_32x128b_warpx4(sfa_t + kb * 4, make_smem_desc(sfa0 + stage * SF_BYTES + kb * 512, 0, 128, 0));
+                    tc_cp_32x128b_warpx4(sfb_t + kb * 4, make_smem_desc(sfb0 + stage * SF_BYTES + kb * 512, 0, 128, 0));
+                }
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const uint64_t ad = make_smem_desc(a0 + stage * A_BYTES + kb * 32, 16, 1024, 2);
+                    const uint64_t bd = make_smem_desc(b0 + stage * C::B_BYTES + kb * 32, 16, 1024, 2);
+                    tc_mma_nvfp4(tmem_base, ad, bd, idesc, sfa_t + kb * 4, sfb_t + kb * 4, (ks | kb) != 0);
+                }
+                tc_commit(&empty[stage]);
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok)
+                tc_commit(acc_full);
+            tc_commit(final_bar);
+            volatile int no_abort = 0;
+            if (!mbar_wait_bounded(final_bar, 0, &no_abort, DRAIN_TIMEOUT_NS))
+                *abort_flag = 1;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        const int nrow = w0 + quarter * 32 + lane;               // output column this lane owns
+        pdl_wait_prerequisites();                               // s_x comes from the quantizer
+        float alpha;
+        {
+            const float sx = *p.s_x;
+            if (p.flags & FLAG_COLLAPSED) {
+                float mx = p.s_w[0];
+                for (int s = 1; s < p.nseg; ++s)
+                    mx = fmaxf(mx, p.s_w[s]);
+                alpha = sx * mx;
+            } else {
+                int seg = 0;
+#pragma unroll
+                for (int s = 0; s < 7; ++s)
+                    seg += (s + 1 < p.nseg && nrow >= p.seg_end[s]) ? 1 : 0;
+                alpha = sx * p.s_w[seg];
+            }
+        }
+        if (mbar_wait_bounded(acc_full, 0, abort_flag, p.timeout_ns)) {
+            tc_fence_after();
+            constexpr int CH = (T < 32) ? T : 32;
+#pragma unroll
+            for (int c0 = 0; c0 < T; c0 += CH) {
+                uint32_t r[CH];
+                __syncwarp();
+                tmem_ld_32x32b<CH>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
+                tmem_ld_wait();
+                if (nrow < p.n) {
+                    if (p.flags & FLAG_F32_OUT) {
+                        float *y = reinterpret_cast<float *>(p.y) + nrow;
+#pragma unroll
+                        for (int i = 0; i < CH; ++i)
+                            if (c0 + i < p.m)
+                                y[static_cast<int64_t>(c0 + i) * p.ldy] = __uint_as_float(r[i]) * alpha;
+                    } else {
+                        __nv_bfloat16 *y = reinterpret_cast<__nv_bfloat16 *>(p.y) + nrow;
+#pragma unroll
+                        for (int i = 0; i < CH; ++i)
+                            if (c0 + i < p.m)
+                                y[static_cast<int64_t>(c0 + i) * p.ldy] =
+                                    __float2bfloat16_rn(__uint_as_float(r[i]) * alpha);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag)
+        atomicCAS(&g_device_error, 0u, 6u /* NVFP4_ERR_TIMEOUT */);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace decode
+}  // namespace nvfp4

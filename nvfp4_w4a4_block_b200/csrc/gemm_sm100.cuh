@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            pdl_wait_prerequisites();            // activation codes come from the preceding kernel
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_mask = 0, issued_phase = 0;
@@ -282,6 +283,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;                    // TMEM lanes this warp may read
         const int row_in_tile = quarter * 32 + lane;
+        pdl_wait_prerequisites();
         const float sx = *p.s_x;
         float swmax = p.s_w[0];
         for (int s = 1; s < p.nseg; ++s)

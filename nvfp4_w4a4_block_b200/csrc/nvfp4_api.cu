@@ -12,10 +12,12 @@
 
 #include <atomic>
 #include <cstdint>
+#include <utility>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/nvfp4.h"
+#include "gemm_decode.cuh"
 #include "gemm_sm100.cuh"
 #include "quantize.cuh"
 
@@ -45,6 +47,26 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
+// Kernel launch; with `pdl` the kernel may start before the previous kernel in
+// the stream finishes (programmatic stream serialization) and must call
+// griddepcontrol.wait before it touches that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t stream, bool pdl,
+                   Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(block));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // One-time per-device set-up: capability check, SM count, kernel attributes,
 // driver entry point for tensor-map encoding.
 nvfp4_status device_setup(int *sms)
@@ -66,7 +88,15 @@ nvfp4_status device_setup(int *sms)
             return d.status;
         }
         if (cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm::SMEM_ALLOC) != cudaSuccess)
+                                 gemm::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Cfg<8>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Cfg<16>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Cfg<32>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Cfg<64>::SMEM_ALLOC) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         if (g_encode == nullptr) {
             cudaDriverEntryPointQueryResult q;
@@ -160,7 +190,8 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
             ap.k = k;
             ap.ldx = ldx;
             ap.partial = partials + s * ga;
-            amax_partial_kernel<<<ga, kQuantThreads, 0, stream>>>(ap);
+            if (launch(amax_partial_kernel, ga, kQuantThreads, 0, stream, false, ap) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
             begin = seg_ends[s];
         }
     }
@@ -181,8 +212,7 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
     qp.partial = partials;
     qp.npartial = ga;
     qp.scale_out = scale_out;
-    quantize_kernel<<<quant_grid(sms, rows, k), kQuantThreads, 0, stream>>>(qp);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch(quantize_kernel, quant_grid(sms, rows, k), kQuantThreads, 0, stream, true, qp));
 }
 
 nvfp4_status make_map(CUtensorMap *map, const void *base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows)
@@ -197,11 +227,60 @@ nvfp4_status make_map(CUtensorMap *map, const void *base, uint64_t inner_bytes, 
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+template <int T>
+nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
+                           const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
+                           const float *seg_gscales, void *y, int64_t ldy, unsigned flags, bool pdl,
+                           cudaStream_t stream)
+{
+    CUtensorMap tw, tx;
+    nvfp4_status st = make_map(&tw, qw, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n), decode::BW);
+    if (st != NVFP4_OK)
+        return st;
+    st = make_map(&tx, qx, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(m), T);
+    if (st != NVFP4_OK)
+        return st;
+    decode::Params p;
+    memset(&p, 0, sizeof p);
+    p.sfw = sfw;
+    p.sfx = sfx;
+    p.m = static_cast<int>(m);
+    p.n = static_cast<int>(n);
+    p.k = static_cast<int>(k);
+    p.atoms_k = k / 64;
+    p.k_stages = static_cast<int>((k + decode::BK - 1) / decode::BK);
+    p.y = y;
+    p.ldy = ldy;
+    p.s_x = s_x;
+    p.s_w = seg_gscales;
+    p.nseg = nseg;
+    for (int s = 0; s < nseg; ++s)
+        p.seg_end[s] = static_cast<int>(seg_ends[s]);
+    p.flags = flags;
+    p.timeout_ns = g_timeout_ns.load();
+    const int grid = static_cast<int>((n + decode::BW - 1) / decode::BW);
+    return cuda_status(launch(decode::nvfp4_gemm_decode_kernel<T>, grid, decode::THREADS, decode::Cfg<T>::SMEM_ALLOC,
+                              stream, pdl, tw, tx, p));
+}
+
+// GEMM + epilogue.  Up to 64 tokens take the swapped decode kernel, more take
+// the persistent 128 x 256 tile kernel.  `pdl` is set only when the preceding
+// kernel in the stream is this library's quantizer, whose early trigger comes
+// after all earlier work has completed (the decode kernel reads weights before
+// it waits on that quantizer).
 nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
                          const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
-                         const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms,
+                         const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms, bool pdl,
                          cudaStream_t stream)
 {
+    if (m <= 8)
+        return launch_decode<8>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
+    if (m <= 16)
+        return launch_decode<16>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
+    if (m <= 32)
+        return launch_decode<32>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
+    if (m <= 64)
+        return launch_decode<64>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
     CUtensorMap ta, tb;
     nvfp4_status st = make_map(&ta, qx, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(m), gemm::BM);
     if (st != NVFP4_OK)
@@ -231,8 +310,7 @@ nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x
     p.timeout_ns = g_timeout_ns.load();
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    gemm::nvfp4_gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_ALLOC, stream>>>(ta, tb, p);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch(gemm::nvfp4_gemm_kernel, grid, gemm::THREADS, gemm::SMEM_ALLOC, stream, pdl, ta, tb, p));
 }
 
 struct WorkspaceLayout {
@@ -379,7 +457,7 @@ nvfp4_status nvfp4_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x,
     int sms = 0;
     if ((st = device_setup(&sms)) != NVFP4_OK)
         return st;
-    return launch_gemm(qx, sfx, s_x, m, qw, sfw, n, k, ends, nseg, seg_gscales, y, ldy, flags, sms,
+    return launch_gemm(qx, sfx, s_x, m, qw, sfw, n, k, ends, nseg, seg_gscales, y, ldy, flags, sms, false,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -417,7 +495,7 @@ nvfp4_status nvfp4_linear_fused(const void *x, int64_t m, int64_t k, int64_t ldx
     if (st != NVFP4_OK)
         return st;
     return launch_gemm(ws + wl.q_off, ws + wl.sf_off, sx, m, qw, sfw, n, k, ends, nseg, seg_gscales, y, ldy, flags,
-                       sms, s);
+                       sms, true, s);
 }
 
 nvfp4_status nvfp4_linear(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,

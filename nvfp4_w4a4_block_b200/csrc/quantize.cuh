@@ -101,6 +101,9 @@ struct AmaxParams {
 
 __global__ void __launch_bounds__(kQuantThreads) amax_partial_kernel(AmaxParams p)
 {
+    // Launched without a programmatic dependency, so everything before it in the
+    // stream has completed; the encode pass may start its prologue right away.
+    pdl_launch_dependents();
     const int64_t upr = p.k >> 3;                          // 16-byte units per row
     const int64_t rows = p.row_end - p.row_begin;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -172,6 +175,12 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
     __shared__ float s_scale[kMaxSeg];
     __shared__ float s_dg[kMaxSeg];
     const int lane = threadIdx.x & 31;
+
+    // Wait for the amax pass (and everything before it), then let the GEMM that
+    // follows start: from this point every kernel before this one has completed,
+    // so the GEMM may stream weights while the codes below are being written.
+    pdl_wait_prerequisites();
+    pdl_launch_dependents();
 
     // Per-segment global scale: given, or amax / 2688 from the amax partials.
     if (threadIdx.x < 32 * p.nseg && (threadIdx.x >> 5) < kMaxSeg) {

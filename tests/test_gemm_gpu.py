@@ -74,6 +74,20 @@ def test_gemm_parity_random(nv, m, n, k, segs):
     assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), bf16_rne_from_f32(y32.cpu().numpy()))
 
 
+@pytest.mark.parametrize("m", [1, 7, 8, 9, 16, 17, 31, 32, 33, 63, 64, 65])
+def test_gemm_token_buckets(nv, m):
+    """Every token-count bucket of the swapped decode kernel (8/16/32/64) and the
+    switch to the tile kernel above 64, with ragged N (200 = 128 + 72) and a
+    partial last K stage (320 = 256 + 64), two segments."""
+    import torch
+    xb, wb, off = W.random_case(20 + m, m, 200, 320, seg_rows=[64, 136])
+    y32, ref, pw = _layer(nv, xb, wb, off, flags=nv.FLAG_F32_OUT)
+    assert_gemm_close(y32.cpu().numpy(), ref["y"], bf16=False)
+    ybf = nv.linear_fused(to_cuda_bf16(xb), pw)
+    torch.cuda.synchronize()
+    assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), bf16_rne_from_f32(y32.cpu().numpy()))
+
+
 def test_gemm_exact_on_representable_operands(nv):
     """E2M1 grid values x power-of-two block magnitudes under power-of-two global
     scales quantize losslessly, so the layer must reproduce X.W^T (fp64 via
