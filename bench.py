@@ -175,6 +175,39 @@ def time_reps(fn, reps, warmup, flush=None):
     return [a.elapsed_time(b) for a, b in out]
 
 
+def capture_graph(fn):
+    """Capture fn() (a sequence of library calls on the current stream) into a
+    CUDA graph so that replays carry no host launch overhead."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()                                 # warm: first-call set-up happens outside capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, reps, per_replay):
+    """Average device time (ms) of one unit when a graph holding per_replay units
+    is replayed back to back `reps` times."""
+    import torch
+    g.replay()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        g.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / (reps * per_replay)
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nvfp4_w4a4_block_b200", "csrc")
@@ -247,19 +280,26 @@ def run_nvfp4(args, rank, world, local_rank):
     wss = {m: torch.empty(nv.workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda") for m in ms}
     torch.cuda.synchronize()
 
-    ctr = [0]
+    # One step = the three calls; call j of the run reads weight copy j % copies.
+    # Steps are replayed from CUDA graphs (one per rotation offset), so the timed
+    # region measures device work, not Python launch overhead.
+    def make_step(first_copy):
+        def step():
+            for j, m in enumerate(ms):
+                nv.linear_fused(xs[m], pws[(first_copy + j) % copies], out=ys[m], ws=wss[m])
+        return step
 
-    def step():
-        for m in ms:
-            pw = pws[ctr[0] % copies]
-            ctr[0] += 1
-            nv.linear_fused(xs[m], pw, out=ys[m], ws=wss[m])
+    n_rot = copies // np.gcd(copies, len(ms))
+    graphs = [capture_graph(make_step((r * len(ms)) % copies)) for r in range(n_rot)]
+
+    def step_i(i):
+        graphs[i % n_rot].replay()
 
     step_bytes = sum(decode_call_bytes(m, n, k) for m in ms)
     launches_per_step = 3 * len(ms)                          # amax, quantize, gemm per call
 
-    for _ in range(args.warmup):
-        step()
+    for i in range(args.warmup):
+        step_i(i)
     torch.cuda.synchronize()
     if nv.get_device_error() != nv.OK:
         raise RuntimeError("device error during warm-up")
@@ -274,15 +314,17 @@ def run_nvfp4(args, rank, world, local_rank):
     s = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s)
-    for _ in range(args.steps):
-        step()
+    for i in range(args.steps):
+        step_i(i)
     e1.record(s)
     # The same step keeps running (untimed) for >= 0.6 s so that the clock
     # sampler sees the load even when the timed region is short.
     t_soak = time.perf_counter()
+    i = 0
     while time.perf_counter() - t_soak < 0.6:
         for _ in range(50):
-            step()
+            step_i(i)
+            i += 1
         torch.cuda.synchronize()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -299,30 +341,32 @@ def run_nvfp4(args, rank, world, local_rank):
     ms_max = float(t.item())
     ms_per_step = ms_max / args.steps
     value = world * step_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    del graphs
 
-    # ---- dominant kernel: the GEMM alone, per M (events on its stream)
+    # ---- dominant kernel: the GEMM alone, per M.  A graph holds `copies` launches
+    # (one per weight copy, so every launch streams from HBM); events on the
+    # replaying stream bracket many replays.
     per_m = {}
     for m in ms:
         qx, sfx, sx = nv.quantize_act(xs[m])
         ym = ys[m]
-        cnt = [0]
 
-        def g():
-            pw = pws[cnt[0] % copies]
-            cnt[0] += 1
-            nv.gemm(qx, sfx, sx, m, pw, out=ym)
+        def gemms():
+            for c in range(copies):
+                nv.gemm(qx, sfx, sx, m, pws[c], out=ym)
 
-        def full():
-            pw = pws[cnt[0] % copies]
-            cnt[0] += 1
-            nv.linear_fused(xs[m], pw, out=ym, ws=wss[m])
+        def calls():
+            for c in range(copies):
+                nv.linear_fused(xs[m], pws[c], out=ym, ws=wss[m])
 
-        tg = time_reps(g, 30, 5)
-        tf = time_reps(full, 30, 5)
+        gg, gc = capture_graph(gemms), capture_graph(calls)
+        tg = time_graph(gg, 20, copies)
+        tf = time_graph(gc, 20, copies)
+        del gg, gc
         gb = decode_call_bytes(m, n, k, gemm_only=True)
         fb = decode_call_bytes(m, n, k)
-        per_m[str(m)] = dict(gemm_us=statistics.median(tg) * 1e3, gemm_gbs=gb / (statistics.median(tg) * 1e-3) / 1e9,
-                             call_us=statistics.median(tf) * 1e3, call_gbs=fb / (statistics.median(tf) * 1e-3) / 1e9,
+        per_m[str(m)] = dict(gemm_us=round(tg * 1e3, 3), gemm_gbs=round(gb / (tg * 1e-3) / 1e9, 1),
+                             call_us=round(tf * 1e3, 3), call_gbs=round(fb / (tf * 1e-3) / 1e9, 1),
                              gemm_bytes=gb, call_bytes=fb)
     gm = per_m[str(mmax)]
     roofline = dict(bound="hbm", kernel="nvfp4_gemm_kernel", workload=f"decode M={mmax}",
@@ -335,6 +379,8 @@ def run_nvfp4(args, rank, world, local_rank):
     hx = {m: xs[m].cpu().pin_memory() for m in ms}
     hy = {m: torch.empty((m, n), dtype=torch.bfloat16).pin_memory() for m in ms}
     dx = {m: torch.empty_like(xs[m]) for m in ms}
+
+    ctr = [0]
 
     def e2e_step():
         for m in ms:
@@ -381,6 +427,7 @@ def run_nvfp4(args, rank, world, local_rank):
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
+        "timing": "timed steps replayed from CUDA graphs (device time, CUDA events on the replay stream)",
         "clocks": clocks,
         "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp4_tflops": round(fp4_peak, 1),
                   "fp4_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} "

@@ -35,10 +35,13 @@ struct DeviceInfo {
     bool ready = false;
     nvfp4_status status = NVFP4_OK;
     int sms = 0;
+    int tile_quant_ctas_per_sm = 1;
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[64];
+thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
+constexpr int64_t kSmallQuantElems = int64_t(1) << 20;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -106,11 +109,17 @@ nvfp4_status device_setup(int *sms)
                 return NVFP4_ERR_CUDA;
             g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
         }
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_tile_kernel, kQuantThreads, 0) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        d.tile_quant_ctas_per_sm = occ > 0 ? occ : 1;
         d.sms = sm;
         d.status = NVFP4_OK;
         d.ready = true;
     }
     *sms = d.sms;
+    g_tile_quant_ctas = d.sms * d.tile_quant_ctas_per_sm;
     return d.status;
 }
 
@@ -174,11 +183,33 @@ int quant_grid(int sms, int64_t rows, int64_t k)
     return static_cast<int>(g < 1 ? 1 : g);
 }
 
-// amax partials (dynamic mode) + encode, rows split into segments.
+// Quantization of [rows, k] (rows split into segments).  Small tensors (at most
+// 2^20 elements, one segment) use one kernel that also reduces the dynamic amax;
+// larger ones run the amax pass (dynamic mode) and the tiled encoder.
 nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx, const int64_t *seg_ends, int nseg,
                              const float *static_scale, float *scale_out, uint8_t *q, uint8_t *sf,
                              uint32_t *partials, int sms, cudaStream_t stream)
 {
+    if (nseg == 1 && rows * k <= kSmallQuantElems) {
+        QuantParams qp;
+        memset(&qp, 0, sizeof qp);
+        qp.x = static_cast<const uint16_t *>(x);
+        qp.rows = rows;
+        qp.k = k;
+        qp.ldx = ldx;
+        qp.q = reinterpret_cast<uint32_t *>(q);
+        qp.sf = sf;
+        qp.rows_pad = (rows + 127) / 128 * 128;
+        qp.kb_pad = ((k / 16) + 3) / 4 * 4;
+        qp.nseg = 1;
+        qp.seg_end[0] = rows;
+        qp.static_scale = static_scale;
+        qp.partial = partials;
+        qp.npartial = 0;
+        qp.scale_out = scale_out;
+        qp.self_amax = static_scale == nullptr ? 1 : 0;
+        return cuda_status(launch(quantize_kernel, quant_grid(sms, rows, k), kQuantThreads, 0, stream, true, qp));
+    }
     const int ga = amax_grid(sms, rows, k);
     if (static_scale == nullptr) {
         int64_t begin = 0;
@@ -195,24 +226,26 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
             begin = seg_ends[s];
         }
     }
-    QuantParams qp;
-    memset(&qp, 0, sizeof qp);
-    qp.x = static_cast<const uint16_t *>(x);
-    qp.rows = rows;
-    qp.k = k;
-    qp.ldx = ldx;
-    qp.q = reinterpret_cast<uint32_t *>(q);
-    qp.sf = sf;
-    qp.rows_pad = (rows + 127) / 128 * 128;
-    qp.kb_pad = ((k / 16) + 3) / 4 * 4;
-    qp.nseg = nseg;
+    TileQuantParams tp;
+    memset(&tp, 0, sizeof tp);
+    tp.x = static_cast<const uint16_t *>(x);
+    tp.rows = rows;
+    tp.k = k;
+    tp.ldx = ldx;
+    tp.q = q;
+    tp.sf = sf;
+    tp.row_tiles = (rows + 127) / 128;
+    tp.col_tiles = k / 64;
+    tp.nseg = nseg;
     for (int s = 0; s < nseg; ++s)
-        qp.seg_end[s] = seg_ends[s];
-    qp.static_scale = static_scale;
-    qp.partial = partials;
-    qp.npartial = ga;
-    qp.scale_out = scale_out;
-    return cuda_status(launch(quantize_kernel, quant_grid(sms, rows, k), kQuantThreads, 0, stream, true, qp));
+        tp.seg_end[s] = seg_ends[s];
+    tp.static_scale = static_scale;
+    tp.partial = partials;
+    tp.npartial = ga;
+    tp.scale_out = scale_out;
+    const int64_t tiles = tp.row_tiles * tp.col_tiles;
+    const int grid = static_cast<int>(tiles < g_tile_quant_ctas ? tiles : g_tile_quant_ctas);
+    return cuda_status(launch(quantize_tile_kernel, grid, kQuantThreads, 0, stream, true, tp));
 }
 
 nvfp4_status make_map(CUtensorMap *map, const void *base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows)

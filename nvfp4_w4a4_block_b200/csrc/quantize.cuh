@@ -168,6 +168,7 @@ struct QuantParams {
     const uint32_t *partial;     // [nseg][npartial] amax partials (dynamic)
     int npartial;
     float *scale_out;            // [nseg]
+    int self_amax;               // dynamic, one segment: each CTA reduces the whole tensor itself
 };
 
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
@@ -182,8 +183,46 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
     pdl_wait_prerequisites();
     pdl_launch_dependents();
 
-    // Per-segment global scale: given, or amax / 2688 from the amax partials.
-    if (threadIdx.x < 32 * p.nseg && (threadIdx.x >> 5) < kMaxSeg) {
+    // Small tensors in dynamic mode: every CTA reduces the whole (L2-resident)
+    // tensor itself, which saves the separate amax launch and its dependency.
+    __shared__ uint32_t s_red[kQuantThreads / 32];
+    if (p.self_amax) {
+        const int64_t upr0 = p.k >> 3;
+        const int64_t total0 = p.rows * upr0;
+        uint32_t b = 0;
+        int64_t r = threadIdx.x / upr0, c = threadIdx.x % upr0;
+        const int64_t sr = blockDim.x / upr0, sc = blockDim.x % upr0;
+        for (int64_t u = threadIdx.x; u < total0; u += blockDim.x) {
+            b = max(b, absmax_bits8(__ldg(reinterpret_cast<const uint4 *>(p.x + r * p.ldx + c * 8))));
+            c += sc;
+            r += sr;
+            if (c >= upr0) {
+                c -= upr0;
+                ++r;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+        if (lane == 0)
+            s_red[threadIdx.x >> 5] = b;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t m = 0;
+            for (int w = 0; w < kQuantThreads / 32; ++w)
+                m = max(m, s_red[w]);
+            float s = __fdiv_rn(__uint_as_float(m << 16), 2688.0f);
+            if (m >= 0x7F80u) {
+                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
+                s = 0.0f;
+            }
+            s_scale[0] = s;
+            s_dg[0] = __fmul_rn(s, 6.0f);
+            if (blockIdx.x == 0)
+                p.scale_out[0] = s;
+        }
+    } else if (threadIdx.x < 32 * p.nseg && (threadIdx.x >> 5) < kMaxSeg) {
+        // Per-segment global scale: given, or amax / 2688 from the amax partials.
         const int seg = threadIdx.x >> 5;
         float s;
         bool finite;
@@ -302,6 +341,173 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
         const int64_t row = p.rows + i / (p.kb_pad >> 2);
         const int64_t kb = (i % (p.kb_pad >> 2)) << 2;
         *reinterpret_cast<uint32_t *>(p.sf + sf_atom_offset(row, kb, p.kb_pad)) = 0u;
+    }
+}
+
+// ------------------------------------------------------------------ encode, tiled
+
+// Large tensors: one CTA iteration owns a tile of 128 rows x 64 columns, i.e.
+// exactly one 512-byte scale atom.  Thread t owns row t/2 and two whole
+// 16-element blocks (64 contiguous input bytes -> 16 bytes of codes, two scale
+// bytes); the atom is assembled in shared memory and leaves as 32 x 16-byte
+// stores, so every output sector is written whole.  The next tile's four 16-byte
+// loads are issued before the current tile is encoded.  Element arithmetic is
+// identical to quantize_kernel (and to the CPU reference).
+struct TileQuantParams {
+    const uint16_t *x;
+    int64_t rows, k, ldx;
+    uint8_t *q;
+    uint8_t *sf;
+    int64_t row_tiles, col_tiles;    // ceil(rows/128), k/64
+    int nseg;
+    int64_t seg_end[kMaxSeg];
+    const float *static_scale;
+    const uint32_t *partial;
+    int npartial;
+    float *scale_out;
+};
+
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// One 16-element block (8 words of bf16 pairs) -> 8 bytes of codes, scale byte.
+__device__ __forceinline__ uint2 encode_block16(const uint32_t (&w)[8], float s, float dg, uint32_t &sb_out)
+{
+    const uint32_t msk = 0x7FFF7FFFu;
+    uint32_t a = __vmaxu2(__vmaxu2(w[0] & msk, w[1] & msk), __vmaxu2(w[2] & msk, w[3] & msk));
+    uint32_t b = __vmaxu2(__vmaxu2(w[4] & msk, w[5] & msk), __vmaxu2(w[6] & msk, w[7] & msk));
+    uint32_t c = __vmaxu2(a, b);
+    const float bmax = __uint_as_float(max(c >> 16, c & 0xFFFFu) << 16);
+    const float sbf = (dg == 0.0f) ? 0.0f : fminf(__fdiv_rn(bmax, dg), 448.0f);
+    const uint32_t sb = f32_to_e4m3(sbf);
+    const float d = __fmul_rn(e4m3_to_f32(sb), s);
+    const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX);
+    const uint64_t rr = (static_cast<uint64_t>(__float_as_uint(r)) << 32) | __float_as_uint(r);
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint64_t pair = (static_cast<uint64_t>(w[i] & 0xFFFF0000u) << 32) | (w[i] << 16);
+        const uint64_t prod = f32x2_mul(pair, rr);
+        v[2 * i] = __uint_as_float(static_cast<uint32_t>(prod));
+        v[2 * i + 1] = __uint_as_float(static_cast<uint32_t>(prod >> 32));
+    }
+    sb_out = sb;
+    return make_uint2(f32x8_to_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]),
+                      f32x8_to_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]));
+}
+
+__global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(TileQuantParams p)
+{
+    __shared__ float s_scale[kMaxSeg];
+    __shared__ float s_dg[kMaxSeg];
+    __shared__ __align__(16) uint32_t s_atom[2][128];
+    const int lane = threadIdx.x & 31;
+
+    pdl_wait_prerequisites();
+    pdl_launch_dependents();
+
+    if (threadIdx.x < 32 * p.nseg && (threadIdx.x >> 5) < kMaxSeg) {
+        const int seg = threadIdx.x >> 5;
+        float s;
+        bool finite;
+        if (p.static_scale != nullptr) {
+            s = p.static_scale[seg];
+            finite = isfinite(s) && s >= 0.0f;
+        } else {
+            uint32_t b = 0;
+            for (int i = lane; i < p.npartial; i += 32)
+                b = max(b, p.partial[seg * p.npartial + i]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+            finite = b < 0x7F80u;
+            s = __fdiv_rn(__uint_as_float(b << 16), 2688.0f);
+        }
+        if (lane == 0) {
+            if (!finite) {
+                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
+                s = 0.0f;
+            }
+            s_scale[seg] = s;
+            s_dg[seg] = __fmul_rn(s, 6.0f);
+            if (blockIdx.x == 0)
+                p.scale_out[seg] = s;
+        }
+    }
+    __syncthreads();
+
+    const int rl = threadIdx.x >> 1;                 // row inside the tile
+    const int half = threadIdx.x & 1;                // columns [32*half, 32*half + 32) of the tile
+    int buf = 0;
+    // Tiles are visited grid-stride in row-tile-major order; (rt, ct) advance by a
+    // fixed step instead of being divided out of the tile index.
+    const int64_t step_r = gridDim.x / p.col_tiles, step_c = gridDim.x % p.col_tiles;
+    int64_t rt = blockIdx.x / p.col_tiles, ct = blockIdx.x % p.col_tiles;
+    auto advance = [&](int64_t &r, int64_t &c) {
+        c += step_c;
+        r += step_r;
+        if (c >= p.col_tiles) {
+            c -= p.col_tiles;
+            ++r;
+        }
+    };
+    auto load = [&](int64_t r, int64_t c, uint4 (&v)[4]) {
+        const int64_t row = r * 128 + rl;
+        if (r < p.row_tiles && row < p.rows) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.ldx + c * 64 + half * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                v[i] = __ldcs(src + i);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                v[i] = make_uint4(0, 0, 0, 0);
+        }
+    };
+    uint4 cur[4];
+    load(rt, ct, cur);
+    while (rt < p.row_tiles) {
+        int64_t rn = rt, cn = ct;
+        advance(rn, cn);
+        uint4 nxt[4];
+        load(rn, cn, nxt);
+
+        const int64_t row = rt * 128 + rl;
+        const bool valid = row < p.rows;
+        int seg = 0;
+#pragma unroll
+        for (int s = 0; s < kMaxSeg - 1; ++s)
+            seg += (s + 1 < p.nseg && row >= p.seg_end[s]) ? 1 : 0;
+        const float s = s_scale[seg], dg = s_dg[seg];
+
+        const uint32_t w0[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+        const uint32_t w1[8] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
+        uint32_t sb0, sb1;
+        const uint2 c0 = encode_block16(w0, s, dg, sb0);
+        const uint2 c1 = encode_block16(w1, s, dg, sb1);
+        if (valid)
+            *reinterpret_cast<uint4 *>(p.q + row * (p.k >> 1) + ct * 32 + half * 16) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+
+        // Scale bytes of blocks (2*half, 2*half+1); the even lane assembles the row's four.
+        const uint32_t mine = valid ? (sb0 | (sb1 << 8)) : 0u;
+        const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, mine, 1);
+        if (half == 0)
+            s_atom[buf][(rl & 31) * 4 + (rl >> 5)] = mine | (other << 16);
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const uint4 v = reinterpret_cast<const uint4 *>(s_atom[buf])[threadIdx.x];
+            *reinterpret_cast<uint4 *>(p.sf + (rt * p.col_tiles + ct) * 512 + threadIdx.x * 16) = v;
+        }
+        buf ^= 1;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            cur[i] = nxt[i];
+        rt = rn;
+        ct = cn;
     }
 }
 

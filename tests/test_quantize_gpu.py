@@ -64,6 +64,27 @@ def test_quantize_random_shapes_dynamic(nv, m, k):
     _compare(nv, x)
 
 
+@pytest.mark.parametrize("m,k", [(1000, 1088), (2049, 1024), (130, 17408), (8192, 128)])
+@pytest.mark.parametrize("static", [None, 0.002])
+def test_quantize_tiled_path_shapes(nv, m, k, static):
+    """Tensors above 2^20 elements take the tiled encoder (128-row x 64-column
+    tiles, whole scale atoms); ragged row tiles leave zero pad scales."""
+    x, _, _ = W.random_case(30, m, 8, k)
+    _compare(nv, x, static)
+
+
+def test_quantize_ties_on_the_tiled_path(nv):
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    rows = []
+    for j in range(-10, 6):
+        blk = np.concatenate([[6.0], ties, -ties, [0.0]]).astype(np.float32) * np.float32(2.0 ** j)
+        rows.append(np.tile(blk, 128))
+    x = W.f32_to_bf16_bits(np.tile(np.stack(rows), (40, 1)))      # 640 x 2048 > 2^20
+    assert x.size > (1 << 20)
+    _compare(nv, x, 2.0 ** -8)
+    _compare(nv, x)
+
+
 @pytest.mark.parametrize("static", [2.0 ** -9, 1e-3, 0.37, 1e-6, 0.0])
 def test_quantize_static_scale(nv, static):
     x, _, _ = W.random_case(4, 200, 8, 512)
