@@ -41,7 +41,8 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[64];
 thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
-constexpr int64_t kSmallQuantElems = int64_t(1) << 20;
+constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder below, tiled encoder above
+constexpr int64_t kSelfAmaxElems = int64_t(1) << 16;     // dynamic scale reduced inside the encoder below
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -190,7 +191,23 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
                              const float *static_scale, float *scale_out, uint8_t *q, uint8_t *sf,
                              uint32_t *partials, int sms, cudaStream_t stream)
 {
+    const int ga = amax_grid(sms, rows, k);
     if (nseg == 1 && rows * k <= kSmallQuantElems) {
+        // Tiny tensors (decode): in dynamic mode every CTA of the single encoder
+        // launch reduces the whole tensor itself (few CTAs, so few redundant reads);
+        // up to 2^20 elements an amax pass precedes the per-unit encoder.
+        const bool self_amax = static_scale == nullptr && rows * k <= kSelfAmaxElems;
+        if (static_scale == nullptr && !self_amax) {
+            AmaxParams ap;
+            ap.x = static_cast<const uint16_t *>(x);
+            ap.row_begin = 0;
+            ap.row_end = rows;
+            ap.k = k;
+            ap.ldx = ldx;
+            ap.partial = partials;
+            if (launch(amax_partial_kernel, ga, kQuantThreads, 0, stream, false, ap) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+        }
         QuantParams qp;
         memset(&qp, 0, sizeof qp);
         qp.x = static_cast<const uint16_t *>(x);
@@ -205,12 +222,14 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
         qp.seg_end[0] = rows;
         qp.static_scale = static_scale;
         qp.partial = partials;
-        qp.npartial = 0;
+        qp.npartial = ga;
         qp.scale_out = scale_out;
-        qp.self_amax = static_scale == nullptr ? 1 : 0;
-        return cuda_status(launch(quantize_kernel, quant_grid(sms, rows, k), kQuantThreads, 0, stream, true, qp));
+        qp.self_amax = self_amax ? 1 : 0;
+        int grid = quant_grid(sms, rows, k);
+        if (self_amax && grid > 16)
+            grid = 16;
+        return cuda_status(launch(quantize_kernel, grid, kQuantThreads, 0, stream, true, qp));
     }
-    const int ga = amax_grid(sms, rows, k);
     if (static_scale == nullptr) {
         int64_t begin = 0;
         for (int s = 0; s < nseg; ++s) {

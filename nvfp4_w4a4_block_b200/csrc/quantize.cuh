@@ -190,16 +190,18 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
         const int64_t upr0 = p.k >> 3;
         const int64_t total0 = p.rows * upr0;
         uint32_t b = 0;
-        int64_t r = threadIdx.x / upr0, c = threadIdx.x % upr0;
-        const int64_t sr = blockDim.x / upr0, sc = blockDim.x % upr0;
-        for (int64_t u = threadIdx.x; u < total0; u += blockDim.x) {
-            b = max(b, absmax_bits8(__ldg(reinterpret_cast<const uint4 *>(p.x + r * p.ldx + c * 8))));
-            c += sc;
-            r += sr;
-            if (c >= upr0) {
-                c -= upr0;
-                ++r;
+        // Four independent 16-byte loads in flight per thread per round.
+        for (int64_t u0 = threadIdx.x; u0 < total0; u0 += 4 * blockDim.x) {
+            uint4 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t u = u0 + j * blockDim.x;
+                v[j] = u < total0 ? __ldg(reinterpret_cast<const uint4 *>(p.x + (u / upr0) * p.ldx + (u % upr0) * 8))
+                                  : make_uint4(0, 0, 0, 0);
             }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                b = max(b, absmax_bits8(v[j]));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
