@@ -1,0 +1,322 @@
+// gemm_pair.cuh -- block-scaled FP4 GEMM on CTA pairs (tcgen05 cta_group::2), sm_100a.
+//
+// Same product and epilogue as gemm_sm100.cuh ("Why Gated DeltaNet Survives 4-Bit
+// Quantization", §2 "NVFP4": the GEMM runs on native 4-bit tensor cores; §6:
+// per-module global scales of a fused GEMM stay separate), organised for the
+// compute-bound prefill regime:
+//
+//   * Two CTAs on neighbouring SMs (a cluster of 2) own a 256 x 256 output tile.
+//     The even CTA issues one M=256, N=256, K=64 block-scaled MMA per 64-deep K
+//     block; each CTA contributes 128 activation rows and 128 weight rows from its
+//     own shared memory and keeps its 128 x 256 half of the accumulator in its own
+//     tensor memory.  Each SM therefore loads 32 KB of codes per 256-deep stage
+//     for 128 x 256 x 256 MACs, a third less than a single-CTA 128 x 256 tile.
+//   * Five 38 KB stages per CTA.  Both CTAs' TMA loads complete on the even CTA's
+//     stage barrier; the even CTA's tcgen05.commit releases the stage in both.
+//   * Eight epilogue warps per CTA drain the accumulator into registers (128
+//     columns each), hand the tensor memory back to the MMA issuer at once, and
+//     only then scale, convert and store -- the next tile's MMAs overlap the
+//     stores.
+//   * Scale factors travel as 512-byte atoms through 3-D tensor maps; both CTAs
+//     load the full 256-row weight-scale block (no multicast of any kind).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace nvfp4 {
+namespace pair {
+
+constexpr int BM = 256;                 // output rows per pair (128 per CTA)
+constexpr int BN = 256;                 // output columns per pair (MMA N)
+constexpr int BK = 256;                 // K elements per stage
+constexpr int KB = BK / 64;
+constexpr int STAGES = 5;
+constexpr int A_BYTES = 128 * BK / 2;   // this CTA's 128 activation rows
+constexpr int B_BYTES = 128 * BK / 2;   // this CTA's 128 weight rows
+constexpr int SFA_BYTES = KB * 512;     // this CTA's 128-row scale block
+constexpr int SFB_BYTES = 2 * KB * 512; // all 256 weight rows' scales
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr uint32_t TX_BYTES = 2 * STAGE_BYTES;   // both CTAs complete on the even CTA's barrier
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr int TMEM_COLS = 512;
+constexpr int TMEM_SFA = BN;
+constexpr int TMEM_SFB = BN + KB * 4;
+constexpr uint64_t DRAIN_TIMEOUT_NS = 1000000000ull;
+
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 3;
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+constexpr int SMEM_ALLOC = OFF_MISC + 64 + 1024;
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(TMEM_SFB + KB * 8 <= TMEM_COLS, "tensor memory budget");
+
+constexpr unsigned FLAG_F32_OUT = 1u;
+constexpr unsigned FLAG_COLLAPSED = 2u;
+
+struct Params {
+    int m, n, k;
+    int tiles_m, tiles_n, k_stages;
+    void *y;
+    int64_t ldy;
+    const float *s_x;
+    const float *s_w;
+    int nseg;
+    int seg_end[8];
+    unsigned flags;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ float col_alpha(const Params &p, float sx, float swmax, int col)
+{
+    if (p.flags & FLAG_COLLAPSED)
+        return sx * swmax;
+    int seg = 0;
+#pragma unroll
+    for (int s = 0; s < 7; ++s)
+        seg += (s + 1 < p.nseg && col >= p.seg_end[s]) ? 1 : 0;
+    return sx * p.s_w[seg];
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                           const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                           const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *empty = full + STAGES;
+    uint64_t *acc_full = full + 2 * STAGES;
+    uint64_t *acc_empty = acc_full + 1;
+    uint64_t *final_bar = acc_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();          // 0: issues the MMAs
+    const int pair_id = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * EPI_WARPS);
+        mbar_init(final_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tm_a);
+        prefetch_tensormap(&tm_b);
+        prefetch_tensormap(&tm_sfa);
+        prefetch_tensormap(&tm_sfb);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    cluster_sync_all();                                // barriers of both CTAs are initialised
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            pdl_wait_prerequisites();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
+                const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(&full[stage], TX_BYTES);
+                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), 0);
+                    tma_load_2d_pair(smem + OFF_A + stage * A_BYTES, &tm_a, ks * (BK / 2),
+                                     mb * BM + static_cast<int>(rank) * 128, bar);
+                    tma_load_2d_pair(smem + OFF_B + stage * B_BYTES, &tm_b, ks * (BK / 2),
+                                     nb * BN + static_cast<int>(rank) * 128, bar);
+                    tma_load_3d_pair(smem + OFF_SFA + stage * SFA_BYTES, &tm_sfa, 0, ks * KB,
+                                     mb * 2 + static_cast<int>(rank), bar);
+                    tma_load_3d_pair(smem + OFF_SFB + stage * SFB_BYTES, &tm_sfb, 0, ks * KB, nb * 2, bar);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // Give copies already issued time to land before the CTA can exit.
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 100000ull) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (rank == 0 && lane == 0) {
+            const uint32_t idesc = make_idesc_nvfp4(BM, BN);
+            const uint32_t sfa_t = tmem_base + TMEM_SFA;
+            const uint32_t sfb_t = tmem_base + TMEM_SFB;
+            const uint32_t a0 = smem_u32(smem + OFF_A), b0 = smem_u32(smem + OFF_B);
+            const uint32_t sfa0 = smem_u32(smem + OFF_SFA), sfb0 = smem_u32(smem + OFF_SFB);
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
+                if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1u, abort_flag, p.timeout_ns))
+                    break;
+                tc_fence_after();
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb) {
+                        tc_cp_32x128b_warpx4_pair(sfa_t + kb * 4,
+                                                  make_smem_desc(sfa0 + stage * SFA_BYTES + kb * 512, 0, 128, 0));
+                        tc_cp_32x128b_warpx4_pair(sfb_t + kb * 8,
+                                                  make_smem_desc(sfb0 + stage * SFB_BYTES + kb * 512, 0, 128, 0));
+                        tc_cp_32x128b_warpx4_pair(
+                            sfb_t + kb * 8 + 4,
+                            make_smem_desc(sfb0 + stage * SFB_BYTES + KB * 512 + kb * 512, 0, 128, 0));
+                    }
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb) {
+                        const uint64_t ad = make_smem_desc(a0 + stage * A_BYTES + kb * 32, 16, 1024, 2);
+                        const uint64_t bd = make_smem_desc(b0 + stage * B_BYTES + kb * 32, 16, 1024, 2);
+                        tc_mma_nvfp4_pair(tmem_base, ad, bd, idesc, sfa_t + kb * 4, sfb_t + kb * 8, (ks | kb) != 0);
+                    }
+                    tc_commit_pair_multicast(&empty[stage], 0x3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                tc_commit_pair_multicast(acc_full, 0x3);
+                acc_phase ^= 1u;
+            }
+            tc_commit_pair(final_bar);
+            volatile int no_abort = 0;
+            if (!mbar_wait_bounded(final_bar, 0, &no_abort, DRAIN_TIMEOUT_NS))
+                *abort_flag = 1;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - 2;                        // 0..7
+        const int quarter = warp & 3;                   // TMEM lanes this warp may read
+        const int col0 = (ew >> 2) * 128;               // this warp's 128 accumulator columns
+        pdl_wait_prerequisites();
+        const float sx = *p.s_x;
+        float swmax = p.s_w[0];
+        for (int s = 1; s < p.nseg; ++s)
+            swmax = fmaxf(swmax, p.s_w[s]);
+        const bool f32_out = (p.flags & FLAG_F32_OUT) != 0;
+        const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
+        uint32_t acc_phase = 0;
+        for (int tile = pair_id; tile < num_tiles; tile += npairs) {
+            const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+            if (!mbar_wait_bounded(acc_full, acc_phase, abort_flag, p.timeout_ns))
+                break;
+            tc_fence_after();
+            uint32_t r[128];
+            __syncwarp();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
+            tmem_ld_32x32b_x32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
+            tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+            tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+            tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_remote(acc_empty_leader);    // the accumulator may be overwritten now
+            acc_phase ^= 1u;
+
+            const int m = mb * BM + static_cast<int>(rank) * 128 + quarter * 32 + lane;
+            if (m < p.m) {
+#pragma unroll
+                for (int c = 0; c < 128; c += 32) {
+                    const int nc = nb * BN + col0 + c;
+                    if (nc >= p.n)
+                        break;
+                    const float a_lo = col_alpha(p, sx, swmax, nc);
+                    const float a_hi = col_alpha(p, sx, swmax, min(nc + 31, p.n - 1));
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        v[i] = __uint_as_float(r[c + i]) *
+                               (a_lo == a_hi ? a_lo : col_alpha(p, sx, swmax, min(nc + i, p.n - 1)));
+                    if (!f32_out) {
+                        __nv_bfloat16 *dst =
+                            reinterpret_cast<__nv_bfloat16 *>(p.y) + static_cast<int64_t>(m) * p.ldy + nc;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (nc + g * 8 < p.n) {
+                                __nv_bfloat162 h0 = __floats2bfloat162_rn(v[g * 8 + 0], v[g * 8 + 1]);
+                                __nv_bfloat162 h1 = __floats2bfloat162_rn(v[g * 8 + 2], v[g * 8 + 3]);
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(v[g * 8 + 4], v[g * 8 + 5]);
+                                __nv_bfloat162 h3 = __floats2bfloat162_rn(v[g * 8 + 6], v[g * 8 + 7]);
+                                uint4 o;
+                                o.x = *reinterpret_cast<uint32_t *>(&h0);
+                                o.y = *reinterpret_cast<uint32_t *>(&h1);
+                                o.z = *reinterpret_cast<uint32_t *>(&h2);
+                                o.w = *reinterpret_cast<uint32_t *>(&h3);
+                                *reinterpret_cast<uint4 *>(dst + g * 8) = o;
+                            }
+                        }
+                    } else {
+                        float *dst = reinterpret_cast<float *>(p.y) + static_cast<int64_t>(m) * p.ldy + nc;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (nc + g * 8 < p.n) {
+                                *reinterpret_cast<float4 *>(dst + g * 8) =
+                                    make_float4(v[g * 8 + 0], v[g * 8 + 1], v[g * 8 + 2], v[g * 8 + 3]);
+                                *reinterpret_cast<float4 *>(dst + g * 8 + 4) =
+                                    make_float4(v[g * 8 + 4], v[g * 8 + 5], v[g * 8 + 6], v[g * 8 + 7]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    cluster_sync_all();                                 // the peer's MMAs and copies are finished
+    if (threadIdx.x == 0 && *abort_flag)
+        atomicCAS(&g_device_error, 0u, 6u /* NVFP4_ERR_TIMEOUT */);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace pair
+}  // namespace nvfp4

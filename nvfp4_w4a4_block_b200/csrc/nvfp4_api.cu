@@ -18,6 +18,7 @@
 
 #include "../../include/nvfp4.h"
 #include "gemm_decode.cuh"
+#include "gemm_pair.cuh"
 #include "gemm_sm100.cuh"
 #include "quantize.cuh"
 
@@ -30,6 +31,7 @@ constexpr int kMaxPartials = 1024;
 constexpr size_t kAlign = 256;
 
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+std::atomic<int> g_use_pair_kernel{1};   // prefill GEMM on CTA pairs (else one CTA per 128 x 256 tile)
 
 struct DeviceInfo {
     bool ready = false;
@@ -42,7 +44,7 @@ std::mutex g_mu;
 DeviceInfo g_dev[64];
 thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
 constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder below, tiled encoder above
-constexpr int64_t kSelfAmaxElems = int64_t(1) << 16;     // dynamic scale reduced inside the encoder below
+constexpr int64_t kSelfAmaxElems = int64_t(1) << 14;     // dynamic scale reduced inside the encoder below
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -93,6 +95,8 @@ nvfp4_status device_setup(int *sms)
         }
         if (cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemm::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(pair::nvfp4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 pair::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Cfg<8>::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -279,6 +283,58 @@ nvfp4_status make_map(CUtensorMap *map, const void *base, uint64_t inner_bytes, 
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Scale atoms as a 3-D tensor: 512-byte atoms (128 x 32-bit), atoms along K,
+// 128-row blocks; a box is 4 atoms (one 256-deep stage) of box_rb row blocks.
+nvfp4_status make_sf_map(CUtensorMap *map, const void *base, uint64_t atoms_k, uint64_t row_blocks, uint32_t box_rb)
+{
+    cuuint64_t dims[3] = {128, atoms_k, row_blocks};
+    cuuint64_t strides[2] = {512, atoms_k * 512};
+    cuuint32_t box[3] = {128, 4, box_rb};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
+                         const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
+                         const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms, bool pdl,
+                         cudaStream_t stream)
+{
+    CUtensorMap ta, tb, tsa, tsb;
+    nvfp4_status st = make_map(&ta, qx, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(m), 128);
+    if (st == NVFP4_OK)
+        st = make_map(&tb, qw, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n), 128);
+    if (st == NVFP4_OK)
+        st = make_sf_map(&tsa, sfx, static_cast<uint64_t>(k / 64), static_cast<uint64_t>((m + 127) / 128), 1);
+    if (st == NVFP4_OK)
+        st = make_sf_map(&tsb, sfw, static_cast<uint64_t>(k / 64), static_cast<uint64_t>((n + 127) / 128), 2);
+    if (st != NVFP4_OK)
+        return st;
+    pair::Params p;
+    memset(&p, 0, sizeof p);
+    p.m = static_cast<int>(m);
+    p.n = static_cast<int>(n);
+    p.k = static_cast<int>(k);
+    p.tiles_m = static_cast<int>((m + pair::BM - 1) / pair::BM);
+    p.tiles_n = static_cast<int>((n + pair::BN - 1) / pair::BN);
+    p.k_stages = static_cast<int>((k + pair::BK - 1) / pair::BK);
+    p.y = y;
+    p.ldy = ldy;
+    p.s_x = s_x;
+    p.s_w = seg_gscales;
+    p.nseg = nseg;
+    for (int s = 0; s < nseg; ++s)
+        p.seg_end[s] = static_cast<int>(seg_ends[s]);
+    p.flags = flags;
+    p.timeout_ns = g_timeout_ns.load();
+    const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+    const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+    return cuda_status(launch(pair::nvfp4_gemm_pair_kernel, static_cast<int>(2 * pairs), pair::THREADS,
+                              pair::SMEM_ALLOC, stream, pdl, ta, tb, tsa, tsb, p));
+}
+
 template <int T>
 nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
                            const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
@@ -333,6 +389,9 @@ nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x
         return launch_decode<32>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
     if (m <= 64)
         return launch_decode<64>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
+    if (g_use_pair_kernel)
+        return launch_pair(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, sms, pdl,
+                           stream);
     CUtensorMap ta, tb;
     nvfp4_status st = make_map(&ta, qx, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(m), gemm::BM);
     if (st != NVFP4_OK)
