@@ -16,7 +16,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/nvfp4.h"
+#include "nvfp4.h"
 #include "gemm_decode.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_sm100.cuh"
