@@ -23,7 +23,8 @@
  * Conventions for every entry point
  *   - All pointers marked "device" are CUDA device (or managed) pointers; the
  *     caller allocates and owns every buffer, including the workspace.  The
- *     library allocates no device memory.
+ *     library allocates no device memory; its only device memory of its own is
+ *     the static scratch array of nvfp4_linear_fused_noalloc (see there).
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream).  No entry point synchronizes, except
  *     nvfp4_get_device_error().
@@ -76,7 +77,8 @@ typedef enum {
     NVFP4_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
     NVFP4_ERR_TIMEOUT = 6,            /* a bounded pipeline wait inside a kernel ran out */
     NVFP4_ERR_WORKSPACE = 7,          /* workspace null or smaller than nvfp4_workspace_bytes() */
-    NVFP4_ERR_UNSUPPORTED_DEVICE = 8  /* current device is not sm_100 */
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 8, /* current device is not sm_100 */
+    NVFP4_ERR_SCRATCH_LIMIT = 9       /* problem too large for nvfp4_linear_fused_noalloc's static scratch */
 } nvfp4_status;
 
 /* Flags for nvfp4_gemm / nvfp4_linear / nvfp4_linear_fused. */
@@ -155,6 +157,35 @@ nvfp4_status nvfp4_linear_fused(const void *x, int64_t m, int64_t k, int64_t ldx
                                 const int64_t *seg_offsets, const float *seg_gscales, int nseg,
                                 void *y, int64_t ldy, unsigned flags,
                                 void *workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* Bytes of the static device scratch behind nvfp4_linear_fused_noalloc.  Every
+ * device that loads this library holds this much device memory until the
+ * process exits. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* The fused layer without a workspace argument, for callers that cannot
+ * allocate device memory: code hosted inside a runtime that owns all device
+ * memory and gives its plugins no allocator, or latency-critical paths where a
+ * cudaMalloc (which may synchronize the device) is not acceptable.  The paper
+ * has no counterpart to this entry point; it is a deployment convenience.
+ *
+ * Arguments, layouts, results and errors are those of nvfp4_linear_fused.  The
+ * activation codes, scales, global scale and amax partials go to a static
+ * device array of NVFP4_NOALLOC_SCRATCH_BYTES inside the library instead of a
+ * caller workspace; a problem whose nvfp4_workspace_bytes(m, n, k) exceeds that
+ * size is rejected with NVFP4_ERR_SCRATCH_LIMIT before anything is enqueued
+ * (at K = 5120 that allows up to about 2900 tokens).
+ *
+ * The first call on a device looks up the array's device address (a one-time
+ * set-up with that device current); make that first call before any stream
+ * capture.  The call allocates nothing.  All calls share the one array and it
+ * keeps the last call's contents; nothing in it needs to start at zero.  Calls
+ * whose work overlaps on the GPU (different streams without ordering between
+ * them) race on the array: order them on one stream. */
+nvfp4_status nvfp4_linear_fused_noalloc(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,
+                                        const uint8_t *qw, const uint8_t *sfw, int64_t n,
+                                        const int64_t *seg_offsets, const float *seg_gscales, int nseg,
+                                        void *y, int64_t ldy, unsigned flags, nvfp4_stream_t stream);
 
 /* Synchronizes `stream`, then returns and clears the current device's error
  * word: NVFP4_ERR_NONFINITE, NVFP4_ERR_TIMEOUT, or NVFP4_OK. */

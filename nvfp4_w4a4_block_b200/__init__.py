@@ -33,6 +33,8 @@ ERR_CUDA = 5
 ERR_TIMEOUT = 6
 ERR_WORKSPACE = 7
 ERR_UNSUPPORTED_DEVICE = 8
+ERR_SCRATCH_LIMIT = 9
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 FLAG_F32_OUT = 0x1
 FLAG_COLLAPSED_MAX_SCALE = 0x2
@@ -40,7 +42,7 @@ MAX_SEGMENTS = 8
 
 EXPORTED = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize_act",
             "nvfp4_pack_weight", "nvfp4_gemm", "nvfp4_linear", "nvfp4_linear_fused", "nvfp4_get_device_error",
-            "nvfp4_set_wait_timeout_ns", "nvfp4_version")
+            "nvfp4_set_wait_timeout_ns", "nvfp4_version", "nvfp4_linear_fused_noalloc")
 
 
 class NVFP4Error(RuntimeError):
@@ -81,6 +83,9 @@ def lib() -> ctypes.CDLL:
                 L.nvfp4_linear_fused.argtypes = [vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, ci, vp, i64, u32, vp,
                                                  sz, vp]
                 L.nvfp4_linear_fused.restype = ci
+                L.nvfp4_linear_fused_noalloc.argtypes = [vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, ci, vp, i64,
+                                                         u32, vp]
+                L.nvfp4_linear_fused_noalloc.restype = ci
                 _lib = L
     return _lib
 
@@ -251,4 +256,23 @@ def linear(x, pw: PackedWeight, act_gscale=None, out=None, flags: int = 0, strea
     st = lib().nvfp4_linear(_ptr(x), m, k, x.stride(0), _ptr(act_gscale), _ptr(pw.q), _ptr(pw.sf), _ptr(pw.gscale),
                             pw.n, _ptr(y), y.stride(0), flags, _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "nvfp4_linear")
+    return y
+
+
+def linear_fused_noalloc(x, pw: PackedWeight, act_gscale=None, out=None, flags: int = 0, stream=None):
+    """linear_fused without a workspace: the library's own static device scratch
+    (NOALLOC_SCRATCH_BYTES per device) holds the activation codes and scales.
+    For callers that cannot allocate device memory.  Calls sharing the scratch
+    must be ordered on one stream; the first call on a device should come before
+    any stream capture."""
+    _check_bf16(x, "x")
+    m, k = x.shape
+    if k != pw.k:
+        raise ValueError("K mismatch")
+    y = _out(m, pw.n, x.device, flags, out)
+    arr, nseg = _seg_array(pw.seg_offsets)
+    st = lib().nvfp4_linear_fused_noalloc(_ptr(x), m, k, x.stride(0), _ptr(act_gscale), _ptr(pw.q), _ptr(pw.sf),
+                                          pw.n, arr, _ptr(pw.gscale), nseg, _ptr(y), y.stride(0), flags,
+                                          _stream(stream))
+    _check(st, "nvfp4_linear_fused_noalloc")
     return y

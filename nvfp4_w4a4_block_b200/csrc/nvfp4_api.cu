@@ -22,6 +22,11 @@
 #include "gemm_sm100.cuh"
 #include "quantize.cuh"
 
+// Device scratch of nvfp4_linear_fused_noalloc (see include/nvfp4.h).  In host
+// code this name is only a stand-in for the device array: its device address is
+// looked up per device with cudaGetSymbolAddress before any kernel gets it.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NVFP4_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 using namespace nvfp4;
@@ -479,6 +484,7 @@ const char *nvfp4_status_string(nvfp4_status st)
     case NVFP4_ERR_TIMEOUT: return "pipeline wait timed out";
     case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
     case NVFP4_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
+    case NVFP4_ERR_SCRATCH_LIMIT: return "problem exceeds the static scratch of nvfp4_linear_fused_noalloc";
     }
     return "unknown status";
 }
@@ -615,6 +621,37 @@ nvfp4_status nvfp4_linear(const void *x, int64_t m, int64_t k, int64_t ldx, cons
 {
     return nvfp4_linear_fused(x, m, k, ldx, act_gscale, qw, sfw, n, nullptr, w_gscale, 1, y, ldy, flags, workspace,
                               ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_linear_fused_noalloc(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,
+                                        const uint8_t *qw, const uint8_t *sfw, int64_t n,
+                                        const int64_t *seg_offsets, const float *seg_gscales, int nseg,
+                                        void *y, int64_t ldy, unsigned flags, nvfp4_stream_t stream)
+{
+    if (m < 0 || k <= 0 || k % 16 != 0)
+        return m < 0 || k <= 0 ? NVFP4_ERR_INVALID_ARG : NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (workspace_layout(m, k).total > NVFP4_NOALLOC_SCRATCH_BYTES)
+        return NVFP4_ERR_SCRATCH_LIMIT;
+    // One-time per-device look-up of the scratch array's device address, made
+    // with that device current.
+    static std::mutex mu;
+    static void *scratch[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return NVFP4_ERR_CUDA;
+    void *ptr = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (scratch[dev] == nullptr) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+                return NVFP4_ERR_CUDA;
+            scratch[dev] = p;
+        }
+        ptr = scratch[dev];
+    }
+    return nvfp4_linear_fused(x, m, k, ldx, act_gscale, qw, sfw, n, seg_offsets, seg_gscales, nseg, y, ldy, flags,
+                              ptr, NVFP4_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream)
