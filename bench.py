@@ -402,7 +402,7 @@ def run_nvfp4(args, rank, world, local_rank):
     workloads = {}
     if rank == 0 and not args.skip_secondary:
         workloads = secondary_workloads(nv, W, peaks, fp4_peak)
-        workloads["decode_per_m"] = per_m
+    workloads["decode_per_m"] = per_m
 
     line = {
         "metric": METRIC,

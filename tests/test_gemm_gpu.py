@@ -156,6 +156,26 @@ def test_gemm_entry_on_prequantized_operands(nv):
     assert torch.equal(y, y2)
 
 
+@pytest.mark.parametrize("m", [1, 5, 8, 16, 31, 32, 64])
+@pytest.mark.parametrize("static", [None, 0.003])
+def test_fused_decode_layer_equals_quantize_then_gemm(nv, m, static):
+    """Up to 64 tokens the layer quantizes the activations inside the GEMM
+    kernel; the result must be bit-identical to quantizing first
+    (nvfp4_quantize_act) and running the GEMM on those codes (nvfp4_gemm)."""
+    import torch
+    xb, wb, off = W.random_case(60 + m, m, 392, 1344, seg_rows=[128, 264])
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    g = None if static is None else torch.tensor([static], dtype=torch.float32, device="cuda")
+    for flags in (nv.FLAG_F32_OUT, 0):
+        fused = nv.linear_fused(x, pw, act_gscale=g, flags=flags)
+        qx, sfx, sx = nv.quantize_act(x, gscale=g)
+        split = nv.gemm(qx, sfx, sx, m, pw, flags=flags)
+        torch.cuda.synchronize()
+        assert nv.get_device_error() == nv.OK
+        assert torch.equal(fused, split)
+
+
 def test_static_activation_scale(nv):
     xb, wb, off = W.random_case(11, 140, 256, 640)
     y, ref, _ = _layer(nv, xb, wb, off, act_static=0.004, flags=nv.FLAG_F32_OUT)
