@@ -359,14 +359,22 @@ def run_nvfp4(args, rank, world, local_rank):
             for c in range(copies):
                 nv.linear_fused(xs[m], pws[c], out=ym, ws=wss[m])
 
-        gg, gc = capture_graph(gemms), capture_graph(calls)
+        static = sx.clone()                 # a calibrated (static) activation scale
+
+        def calls_static():
+            for c in range(copies):
+                nv.linear_fused(xs[m], pws[c], act_gscale=static, out=ym, ws=wss[m])
+
+        gg, gc, gs = capture_graph(gemms), capture_graph(calls), capture_graph(calls_static)
         tg = time_graph(gg, 20, copies)
         tf = time_graph(gc, 20, copies)
-        del gg, gc
+        ts = time_graph(gs, 20, copies)
+        del gg, gc, gs
         gb = decode_call_bytes(m, n, k, gemm_only=True)
         fb = decode_call_bytes(m, n, k)
         per_m[str(m)] = dict(gemm_us=round(tg * 1e3, 3), gemm_gbs=round(gb / (tg * 1e-3) / 1e9, 1),
                              call_us=round(tf * 1e3, 3), call_gbs=round(fb / (tf * 1e-3) / 1e9, 1),
+                             call_static_scale_us=round(ts * 1e3, 3),
                              gemm_bytes=gb, call_bytes=fb)
     gm = per_m[str(mmax)]
     roofline = dict(bound="hbm", kernel="nvfp4_gemm_kernel", workload=f"decode M={mmax}",

@@ -26,7 +26,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include "quantize.cuh"
 #include "sm100_ptx.cuh"
 
 namespace nvfp4 {
@@ -234,282 +233,6 @@ __global__ void __launch_bounds__(THREADS, 2)
             }
         }
         if (mbar_wait_bounded(acc_full, 0, abort_flag, p.timeout_ns)) {
-            tc_fence_after();
-            constexpr int CH = (T < 32) ? T : 32;
-#pragma unroll
-            for (int c0 = 0; c0 < T; c0 += CH) {
-                uint32_t r[CH];
-                __syncwarp();
-                tmem_ld_32x32b<CH>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
-                tmem_ld_wait();
-                if (nrow < p.n) {
-                    if (p.flags & FLAG_F32_OUT) {
-                        float *y = reinterpret_cast<float *>(p.y) + nrow;
-#pragma unroll
-                        for (int i = 0; i < CH; ++i)
-                            if (c0 + i < p.m)
-                                y[static_cast<int64_t>(c0 + i) * p.ldy] = __uint_as_float(r[i]) * alpha;
-                    } else {
-                        __nv_bfloat16 *y = reinterpret_cast<__nv_bfloat16 *>(p.y) + nrow;
-#pragma unroll
-                        for (int i = 0; i < CH; ++i)
-                            if (c0 + i < p.m)
-                                y[static_cast<int64_t>(c0 + i) * p.ldy] =
-                                    __float2bfloat16_rn(__uint_as_float(r[i]) * alpha);
-                    }
-                }
-            }
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0 && *abort_flag)
-        atomicCAS(&g_device_error, 0u, 6u /* NVFP4_ERR_TIMEOUT */);
-    if (warp == 1) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
-    }
-}
-
-}  // namespace decode
-}  // namespace nvfp4
-
-// ---------------------------------------------------------------------------
-// The whole layer in one kernel for few tokens: activation quantization fused
-// into the GEMM (the fused decode row of the design: the paper's §9 attributes
-// the remaining decode loss to small-batch activation quantization).
-//
-// The four epilogue warps are idle while the mainloop runs, so they quantize:
-// for every 256-deep stage they read the T x 256 bf16 activation slice (L2
-// resident), encode it with exactly the arithmetic of the standalone quantizer
-// (encode_block16), and write the codes in the 128-byte-swizzled layout a TMA
-// load would have produced and the scale bytes in the 512-byte atom layout,
-// straight into the stage's shared-memory B operand.  The weight stages stream
-// by TMA from the first cycle.  In dynamic mode the global scale comes from the
-// amax partials of a preceding amax pass (the only other launch); the
-// quantizing warps wait for it with griddepcontrol.wait while the weights
-// already stream.  Afterwards the same warps run the epilogue.
-// ---------------------------------------------------------------------------
-namespace nvfp4 {
-namespace decode {
-
-struct FusedParams {
-    const uint16_t *x;           // bf16 activations [m, k]
-    int64_t ldx;
-    const uint8_t *sfw;
-    int m, n, k;
-    int64_t atoms_k;
-    int k_stages;
-    void *y;
-    int64_t ldy;
-    const float *act_scale;      // static global scale, or nullptr (dynamic)
-    const uint32_t *partial;     // amax partials of the preceding pass (dynamic)
-    int npartial;
-    float *scale_out;            // receives the activation global scale used
-    const float *s_w;
-    int nseg;
-    int seg_end[8];
-    unsigned flags;
-    uint64_t timeout_ns;
-};
-
-template <int T>
-__global__ void __launch_bounds__(THREADS, 2)
-    nvfp4_linear_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const FusedParams p)
-{
-    using C = Cfg<T>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *empty = full + C::STAGES;
-    uint64_t *acc_full = full + 2 * C::STAGES;
-    uint64_t *final_bar = acc_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int w0 = blockIdx.x * BW;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], 1 + 4);          // weight copies + the four quantizing warps
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(acc_full, 1);
-        mbar_init(final_bar, 1);
-        *abort_flag = 0;
-        fence_barrier_init();
-        prefetch_tensormap(&tm_w);
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-
-    if (warp == 0) {
-        // ------------------------------------------------------------ weight producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued = 0;
-            for (int ks = 0; ks < p.k_stages; ++ks) {
-                if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns))
-                    break;
-                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
-                mbar_arrive_expect_tx(&full[stage], A_BYTES + nkb * 512);
-                tma_load_2d(smem + C::OFF_A + stage * A_BYTES, &tm_w, ks * (BK / 2), w0, &full[stage]);
-                bulk_load(smem + C::OFF_SFA + stage * SF_BYTES,
-                          p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512, nkb * 512,
-                          &full[stage]);
-                issued = ks + 1;
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            for (int j = 0; j < min(C::STAGES, issued); ++j) {
-                const int ks = issued - 1 - j;
-                volatile int no_abort = 0;
-                if (!mbar_wait_bounded(&full[ks % C::STAGES], static_cast<uint32_t>((ks / C::STAGES) & 1), &no_abort,
-                                       DRAIN_TIMEOUT_NS))
-                    *abort_flag = 1;
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc_nvfp4(BW, T);
-            const uint32_t sfa_t = tmem_base + C::TMEM_SFA;
-            const uint32_t sfb_t = tmem_base + C::TMEM_SFB;
-            const uint32_t a0 = smem_u32(smem + C::OFF_A), b0 = smem_u32(smem + C::OFF_B);
-            const uint32_t sfa0 = smem_u32(smem + C::OFF_SFA), sfb0 = smem_u32(smem + C::OFF_SFB);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int ks = 0; ks < p.k_stages; ++ks) {
-                if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
-                for (int kb = 0; kb < nkb; ++kb) {
-                    tc_cp_32x128b_warpx4(sfa_t + kb * 4, make_smem_desc(sfa0 + stage * SF_BYTES + kb * 512, 0, 128, 0));
-                    tc_cp_32x128b_warpx4(sfb_t + kb * 4, make_smem_desc(sfb0 + stage * SF_BYTES + kb * 512, 0, 128, 0));
-                }
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const uint64_t ad = make_smem_desc(a0 + stage * A_BYTES + kb * 32, 16, 1024, 2);
-                    const uint64_t bd = make_smem_desc(b0 + stage * C::B_BYTES + kb * 32, 16, 1024, 2);
-                    tc_mma_nvfp4(tmem_base, ad, bd, idesc, sfa_t + kb * 4, sfb_t + kb * 4, (ks | kb) != 0);
-                }
-                tc_commit(&empty[stage]);
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (ok)
-                tc_commit(acc_full);
-            tc_commit(final_bar);
-            volatile int no_abort = 0;
-            if (!mbar_wait_bounded(final_bar, 0, &no_abort, DRAIN_TIMEOUT_NS))
-                *abort_flag = 1;
-        }
-    } else {
-        // ------------------------------------------------------------ quantizer, then epilogue
-        const int qt = threadIdx.x - 64;                           // 0..127
-        // Activation global scale: the static one, or amax/2688 from the amax pass.
-        float s;
-        bool finite;
-        if (p.act_scale != nullptr) {
-            s = *p.act_scale;
-            finite = isfinite(s) && s >= 0.0f;
-        } else {
-            pdl_wait_prerequisites();
-            uint32_t b = 0;
-            for (int i = lane; i < p.npartial; i += 32)
-                b = max(b, p.partial[i]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
-            finite = b < 0x7F80u;
-            s = __fdiv_rn(__uint_as_float(b << 16), 2688.0f);
-        }
-        if (!finite)
-            s = 0.0f;
-        if (qt == 0) {
-            if (!finite)
-                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
-            if (blockIdx.x == 0 && p.scale_out != nullptr)
-                *p.scale_out = s;
-        }
-        const float dg = __fmul_rn(s, 6.0f);
-
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        for (int ks = 0; ks < p.k_stages && ok; ++ks) {
-            if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
-                ok = false;
-                break;
-            }
-            const int nblk = min(KB, static_cast<int>(p.atoms_k) - ks * KB) * 4;    // valid 16-element blocks
-            uint8_t *bsm = smem + C::OFF_B + stage * C::B_BYTES;
-            uint8_t *ssm = smem + C::OFF_SFB + stage * SF_BYTES;
-#pragma unroll
-            for (int j = 0; j < T / 8; ++j) {
-                const int idx = qt + j * 128;                          // (token, block) = (idx/16, idx%16)
-                const int t = idx >> 4, b = idx & 15;
-                uint2 codes = make_uint2(0, 0);
-                uint32_t sb = 0;
-                if (t < p.m && b < nblk) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(t) * p.ldx +
-                                                                       static_cast<int64_t>(ks) * BK + b * 16);
-                    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                    codes = encode_block16(w, s, dg, sb);
-                }
-                // Codes: row t, 16-byte chunk b/2 (128-byte swizzle: chunk ^ (t % 8)), half b%2.
-                *reinterpret_cast<uint2 *>(bsm + t * 128 + ((((b >> 1) ^ (t & 7)) << 4) | ((b & 1) << 3))) = codes;
-                // Scale byte: atom b/4, row t, column b%4.
-                ssm[(b >> 2) * 512 + (t & 31) * 16 + (t >> 5) * 4 + (b & 3)] = static_cast<uint8_t>(sb);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&full[stage]);
-            if (++stage == C::STAGES) {
-                stage = 0;
-                phase ^= 1u;
-            }
-        }
-
-        // epilogue
-        const int quarter = warp & 3;
-        const int nrow = w0 + quarter * 32 + lane;
-        float alpha;
-        {
-            if (p.flags & FLAG_COLLAPSED) {
-                float mx = p.s_w[0];
-                for (int i = 1; i < p.nseg; ++i)
-                    mx = fmaxf(mx, p.s_w[i]);
-                alpha = s * mx;
-            } else {
-                int seg = 0;
-#pragma unroll
-                for (int i = 0; i < 7; ++i)
-                    seg += (i + 1 < p.nseg && nrow >= p.seg_end[i]) ? 1 : 0;
-                alpha = s * p.s_w[seg];
-            }
-        }
-        if (ok && mbar_wait_bounded(acc_full, 0, abort_flag, p.timeout_ns)) {
             tc_fence_after();
             constexpr int CH = (T < 32) ? T : 32;
 #pragma unroll

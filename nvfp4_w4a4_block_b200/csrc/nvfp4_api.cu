@@ -109,14 +109,6 @@ nvfp4_status device_setup(int *sms)
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Cfg<32>::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode::Cfg<64>::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(decode::nvfp4_linear_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode::Cfg<8>::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(decode::nvfp4_linear_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode::Cfg<16>::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(decode::nvfp4_linear_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode::Cfg<32>::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(decode::nvfp4_linear_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Cfg<64>::SMEM_ALLOC) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         if (g_encode == nullptr) {
@@ -437,60 +429,6 @@ nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x
     return cuda_status(launch(gemm::nvfp4_gemm_kernel, grid, gemm::THREADS, gemm::SMEM_ALLOC, stream, pdl, ta, tb, p));
 }
 
-// The whole layer for up to 64 tokens: [amax pass] + one kernel that quantizes the
-// activations into its own shared-memory stages while it streams the weights.
-// In dynamic mode the kernel follows the amax pass with a programmatic dependency
-// (the amax pass starts only after all earlier work, so the weights it streams
-// before waiting are complete); with a static scale it is launched plainly.
-template <int T>
-nvfp4_status launch_linear_decode(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,
-                                  const uint8_t *qw, const uint8_t *sfw, int64_t n, const int64_t *seg_ends, int nseg,
-                                  const float *seg_gscales, void *y, int64_t ldy, unsigned flags, uint32_t *partials,
-                                  float *scale_out, int sms, cudaStream_t stream)
-{
-    CUtensorMap tw;
-    nvfp4_status st = make_map(&tw, qw, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n), decode::BW);
-    if (st != NVFP4_OK)
-        return st;
-    const int ga = amax_grid(sms, m, k);
-    if (act_gscale == nullptr) {
-        AmaxParams ap;
-        ap.x = static_cast<const uint16_t *>(x);
-        ap.row_begin = 0;
-        ap.row_end = m;
-        ap.k = k;
-        ap.ldx = ldx;
-        ap.partial = partials;
-        if (launch(amax_partial_kernel, ga, kQuantThreads, 0, stream, false, ap) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-    }
-    decode::FusedParams p;
-    memset(&p, 0, sizeof p);
-    p.x = static_cast<const uint16_t *>(x);
-    p.ldx = ldx;
-    p.sfw = sfw;
-    p.m = static_cast<int>(m);
-    p.n = static_cast<int>(n);
-    p.k = static_cast<int>(k);
-    p.atoms_k = k / 64;
-    p.k_stages = static_cast<int>((k + decode::BK - 1) / decode::BK);
-    p.y = y;
-    p.ldy = ldy;
-    p.act_scale = act_gscale;
-    p.partial = partials;
-    p.npartial = ga;
-    p.scale_out = scale_out;
-    p.s_w = seg_gscales;
-    p.nseg = nseg;
-    for (int s = 0; s < nseg; ++s)
-        p.seg_end[s] = static_cast<int>(seg_ends[s]);
-    p.flags = flags;
-    p.timeout_ns = g_timeout_ns.load();
-    const int grid = static_cast<int>((n + decode::BW - 1) / decode::BW);
-    return cuda_status(launch(decode::nvfp4_linear_decode_kernel<T>, grid, decode::THREADS, decode::Cfg<T>::SMEM_ALLOC,
-                              stream, act_gscale == nullptr, tw, p));
-}
-
 struct WorkspaceLayout {
     size_t q_off, sf_off, scale_off, total;
 };
@@ -668,20 +606,6 @@ nvfp4_status nvfp4_linear_fused(const void *x, int64_t m, int64_t k, int64_t ldx
         return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float *sx = reinterpret_cast<float *>(ws + wl.scale_off);
-    if (m <= 64) {
-        uint32_t *partials = reinterpret_cast<uint32_t *>(ws);
-#define NVFP4_DECODE(T_)                                                                                               \
-    return launch_linear_decode<T_>(x, m, k, ldx, act_gscale, qw, sfw, n, ends, nseg, seg_gscales, y, ldy, flags,      \
-                                    partials, sx, sms, s)
-        if (m <= 8)
-            NVFP4_DECODE(8);
-        if (m <= 16)
-            NVFP4_DECODE(16);
-        if (m <= 32)
-            NVFP4_DECODE(32);
-        NVFP4_DECODE(64);
-#undef NVFP4_DECODE
-    }
     int64_t end = m;
     st = launch_quantize(x, m, k, ldx, &end, 1, act_gscale, sx, ws + wl.q_off, ws + wl.sf_off,
                          reinterpret_cast<uint32_t *>(ws), sms, s);

@@ -158,10 +158,10 @@ def test_gemm_entry_on_prequantized_operands(nv):
 
 @pytest.mark.parametrize("m", [1, 5, 8, 16, 31, 32, 64])
 @pytest.mark.parametrize("static", [None, 0.003])
-def test_fused_decode_layer_equals_quantize_then_gemm(nv, m, static):
-    """Up to 64 tokens the layer quantizes the activations inside the GEMM
-    kernel; the result must be bit-identical to quantizing first
-    (nvfp4_quantize_act) and running the GEMM on those codes (nvfp4_gemm)."""
+def test_layer_equals_quantize_then_gemm(nv, m, static):
+    """The whole layer (nvfp4_linear_fused, which chains the quantizer and the
+    GEMM with programmatic dependent launch) is bit-identical to quantizing
+    first (nvfp4_quantize_act) and running the GEMM on those codes (nvfp4_gemm)."""
     import torch
     xb, wb, off = W.random_case(60 + m, m, 392, 1344, seg_rows=[128, 264])
     x = to_cuda_bf16(xb)
