@@ -57,6 +57,9 @@ def _load():
         lib.or_linear_rows.argtypes = [vp, vp, f32, vp, i64, vp, vp, vp, i64, i64, vp]
         lib.or_linear_rows.restype = None
         lib.or_num_threads.argtypes, lib.or_num_threads.restype = [], ctypes.c_int
+        lib.or_bf16_from_f64.argtypes, lib.or_bf16_from_f64.restype = [f64], ctypes.c_uint16
+        lib.or_dequantize_bf16.argtypes, lib.or_dequantize_bf16.restype = [vp, vp, i64, i64, vp, vp], None
+        lib.or_harmonize.argtypes, lib.or_harmonize.restype = [vp, i64, i64, vp, ctypes.c_int, vp], f32
         _lib = lib
     return _lib
 
@@ -168,6 +171,41 @@ def sf_to_physical(sf: np.ndarray, k: int) -> np.ndarray:
     phys = np.zeros(sf_physical_bytes(rows, k), dtype=np.uint8)
     _load().or_sf_to_physical(_ptr(sf), rows, k, _ptr(phys))
     return phys
+
+
+def import_scales(sf_linear: np.ndarray, k: int) -> np.ndarray:
+    """Checkpoint import (R16): a linear-layout block-scale matrix [rows, k/16]
+    is the logical matrix; its physical form is the R10 scatter of it."""
+    return sf_to_physical(sf_linear, k)
+
+
+def bf16_from_f64(v: float) -> int:
+    """Bits of the bf16 nearest to v (ties to the even significand)."""
+    return int(_load().or_bf16_from_f64(float(v)))
+
+
+def dequantize_bf16(q: np.ndarray, sf: np.ndarray, row_scale) -> np.ndarray:
+    """Packed codes + logical scales -> bf16 bit patterns [rows, k] (R14)."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    rows = q.shape[0]
+    k = q.shape[1] * 2
+    rs = np.ascontiguousarray(np.broadcast_to(np.asarray(row_scale, dtype=np.float32), (rows,)))
+    out = np.zeros((rows, k), dtype=np.uint16)
+    if rows:
+        _load().or_dequantize_bf16(_ptr(q), _ptr(sf), rows, k, _ptr(rs), _ptr(out))
+    return out
+
+
+def harmonize(sf: np.ndarray, seg_offsets: Sequence[int], seg_scale: Sequence[float]) -> tuple:
+    """Fold per-module global scales into the block scales of a fused weight (R15).
+    Returns (new logical sf [rows, k/16], shared global scale)."""
+    out = np.array(sf, dtype=np.uint8, copy=True, order="C")
+    rows, nblk = out.shape
+    offs = np.ascontiguousarray(np.asarray(seg_offsets, dtype=np.int64))
+    sc = np.ascontiguousarray(np.asarray(seg_scale, dtype=np.float32))
+    shared = _load().or_harmonize(_ptr(out), rows, nblk * 16, _ptr(offs), len(sc), _ptr(sc))
+    return out, np.float32(shared)
 
 
 # --- GEMM ------------------------------------------------------------------

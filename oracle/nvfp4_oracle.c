@@ -41,6 +41,21 @@
  *      Pad bytes are 0.
  *  R11 GEMM: exact fp64 sum over k of value(code_x)*sd_x * value(code_w)*sd_w,
  *      then times s_x and times s_w of the column's segment, in fp64.
+ *  R14 Dequantization to bf16 (the model card's "expand to BF16"): each element
+ *      is value(code) * value(block scale) * s, a product that is exact in fp64
+ *      (2 + 4 + 24 significant bits), rounded once to the nearest bf16, ties to
+ *      the even significand.
+ *  R15 Harmonization of a fused group ("Why Gated DeltaNet Survives 4-Bit
+ *      Quantization", §6, the checkpoint-side repair): the group's shared global
+ *      scale is the largest of its modules' scales, s_shared = max_i s_i, and
+ *      every block scale of module i becomes E4M3(value(sb) * (s_i / s_shared)),
+ *      ratio and product in fp32 round-to-nearest, then R5's rounding.  With the
+ *      largest scale as the shared one every ratio is <= 1, so no folded scale
+ *      can pass 448 and the re-rounding error stays within E4M3's half ulp
+ *      (2^-4 relative in the normal range; the paper reports <= 6.2%).
+ *  R16 Checkpoint import: a linear-layout block-scale matrix [rows, K/16]
+ *      (one E4M3 byte per block, rows contiguous) is the logical matrix that
+ *      R10 scatters; the packed codes need no change (same nibble order, R9).
  *
  * Build: gcc -O2 -fopenmp -fPIC -shared -ffp-contract=off -fno-fast-math
  */
@@ -299,3 +314,85 @@ int or_num_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------ */
+/* bf16 rounding and dequantization to bf16 (R14)                            */
+/* ------------------------------------------------------------------------ */
+
+/* Nearest bf16 (8 significant bits, fp32's exponent range, subnormals kept) to
+ * a double; a tie goes to the even significand; a magnitude at or past the
+ * largest finite value plus half an ulp becomes infinity.  Returns the bits. */
+uint16_t or_bf16_from_f64(double v)
+{
+    if (isnan(v))
+        return 0x7FC0u;
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7F80u);
+    int e;
+    frexp(a, &e);                        /* a in [2^(e-1), 2^e) */
+    int qexp = e - 8;                    /* spacing of 8-significant-bit values there */
+    if (qexp < -133)                     /* subnormal spacing 2^-126 * 2^-7 */
+        qexp = -133;
+    double r = nearbyint(ldexp(a, -qexp));   /* exact scaling; nearest integer, ties to even */
+    double rounded = ldexp(r, qexp);
+    if (rounded >= ldexp(1.0, 128))
+        return (uint16_t)(sign | 0x7F80u);
+    float f = (float)rounded;            /* exact: at most 8 significant bits, inside fp32's range */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFFu));
+}
+
+/* Dequantize packed rows to bf16: out[r, j] = bf16(value(code) * value(sf) * s_r). */
+void or_dequantize_bf16(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t k, const float *row_scale,
+                        uint16_t *out)
+{
+    const int64_t nblk = k / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            uint8_t byte = q[r * (k / 2) + j / 2];
+            uint32_t code = (j & 1) ? (byte >> 4) : (byte & 15u);
+            double exact = or_e2m1_value(code) * or_e4m3_value(sf[r * nblk + j / 16]) * (double)row_scale[r];
+            out[r * k + j] = or_bf16_from_f64(exact);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Harmonization of a fused group (R15)                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Rewrites the logical block scales sf[rows, k/16] of a weight whose row
+ * segments [seg_offsets[i], seg_offsets[i+1]) carry global scales seg_scale[i]
+ * so that the whole weight uses one global scale, which is returned.  A
+ * non-finite or negative scale leaves sf untouched and returns NaN; an all-zero
+ * group (shared scale 0) is left as it is. */
+float or_harmonize(uint8_t *sf, int64_t rows, int64_t k, const int64_t *seg_offsets, int nseg,
+                   const float *seg_scale)
+{
+    (void)rows;
+    float shared = 0.0f;
+    for (int i = 0; i < nseg; ++i) {
+        if (!isfinite(seg_scale[i]) || seg_scale[i] < 0.0f)
+            return NAN;
+        if (seg_scale[i] > shared)
+            shared = seg_scale[i];
+    }
+    if (shared == 0.0f)
+        return shared;
+    const int64_t nblk = k / 16;
+    for (int i = 0; i < nseg; ++i) {
+        float ratio = seg_scale[i] / shared;                 /* fp32, <= 1 */
+        for (int64_t r = seg_offsets[i]; r < seg_offsets[i + 1]; ++r)
+            for (int64_t c = 0; c < nblk; ++c) {
+                float folded = (float)or_e4m3_value(sf[r * nblk + c]) * ratio;   /* fp32 product */
+                sf[r * nblk + c] = (uint8_t)or_e4m3_encode(folded);
+            }
+    }
+    return shared;
+}
+
