@@ -136,44 +136,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
-        if (lane == 0) {
-            pdl_wait_prerequisites();
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
-                const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
-                for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
+        // The whole warp walks the schedule (so every operand below is
+        // warp-uniform); one elected lane issues the copies.
+        pdl_wait_prerequisites();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        const uint32_t bar0 = map_to_rank(smem_u32(&full[0]), 0);
+        for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
+            const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+            const int row_a = mb * BM + static_cast<int>(rank) * 128;
+            const int row_b = nb * BN + static_cast<int>(rank) * 128;
+            for (int ks = 0; ks < p.k_stages; ++ks) {
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns));
+                if (!ok)
+                    break;
+                const uint32_t bar = bar0 + stage * 8;
+                if (elect_one()) {
                     if (rank == 0)
                         mbar_arrive_expect_tx(&full[stage], TX_BYTES);
-                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), 0);
-                    tma_load_2d_pair(smem + OFF_A + stage * A_BYTES, &tm_a, ks * (BK / 2),
-                                     mb * BM + static_cast<int>(rank) * 128, bar);
-                    tma_load_2d_pair(smem + OFF_B + stage * B_BYTES, &tm_b, ks * (BK / 2),
-                                     nb * BN + static_cast<int>(rank) * 128, bar);
+                    tma_load_2d_pair(smem + OFF_A + stage * A_BYTES, &tm_a, ks * (BK / 2), row_a, bar);
+                    tma_load_2d_pair(smem + OFF_B + stage * B_BYTES, &tm_b, ks * (BK / 2), row_b, bar);
                     tma_load_3d_pair(smem + OFF_SFA + stage * SFA_BYTES, &tm_sfa, 0, ks * KB,
                                      mb * 2 + static_cast<int>(rank), bar);
                     tma_load_3d_pair(smem + OFF_SFB + stage * SFB_BYTES, &tm_sfb, 0, ks * KB, nb * 2, bar);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            if (!ok) {
-                // Give copies already issued time to land before the CTA can exit.
-                const uint64_t t0 = global_timer_ns();
-                while (global_timer_ns() - t0 < 100000ull) {
-                }
+        }
+        if (!ok) {
+            // Give copies already issued time to land before the CTA can exit.
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 100000ull) {
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (even CTA)
-        if (rank == 0 && lane == 0) {
+        // The whole warp runs the loop; an elected lane issues the scale copies,
+        // the MMAs and the commits (always the same lane, lane 0, since the warp
+        // is converged there, so one thread's commits cover all its MMAs).
+        if (rank == 0) {
             const uint32_t idesc = make_idesc_nvfp4(BM, BN);
             const uint32_t sfa_t = tmem_base + TMEM_SFA;
             const uint32_t sfb_t = tmem_base + TMEM_SFB;
@@ -183,32 +189,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
-                if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1u, abort_flag, p.timeout_ns))
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_empty, acc_phase ^ 1u, abort_flag, p.timeout_ns));
+                if (!ok)
                     break;
                 tc_fence_after();
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
-                        ok = false;
+                    ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns));
+                    if (!ok)
                         break;
-                    }
                     tc_fence_after();
+                    const uint32_t sfa_s = sfa0 + stage * SFA_BYTES, sfb_s = sfb0 + stage * SFB_BYTES;
+                    const uint32_t a_s = a0 + stage * A_BYTES, b_s = b0 + stage * B_BYTES;
+                    if (elect_one()) {
 #pragma unroll
-                    for (int kb = 0; kb < KB; ++kb) {
-                        tc_cp_32x128b_warpx4_pair(sfa_t + kb * 4,
-                                                  make_smem_desc(sfa0 + stage * SFA_BYTES + kb * 512, 0, 128, 0));
-                        tc_cp_32x128b_warpx4_pair(sfb_t + kb * 8,
-                                                  make_smem_desc(sfb0 + stage * SFB_BYTES + kb * 512, 0, 128, 0));
-                        tc_cp_32x128b_warpx4_pair(
-                            sfb_t + kb * 8 + 4,
-                            make_smem_desc(sfb0 + stage * SFB_BYTES + KB * 512 + kb * 512, 0, 128, 0));
-                    }
+                        for (int kb = 0; kb < KB; ++kb) {
+                            tc_cp_32x128b_warpx4_pair(sfa_t + kb * 4, make_smem_desc(sfa_s + kb * 512, 0, 128, 0));
+                            tc_cp_32x128b_warpx4_pair(sfb_t + kb * 8, make_smem_desc(sfb_s + kb * 512, 0, 128, 0));
+                            tc_cp_32x128b_warpx4_pair(sfb_t + kb * 8 + 4,
+                                                      make_smem_desc(sfb_s + KB * 512 + kb * 512, 0, 128, 0));
+                        }
 #pragma unroll
-                    for (int kb = 0; kb < KB; ++kb) {
-                        const uint64_t ad = make_smem_desc(a0 + stage * A_BYTES + kb * 32, 16, 1024, 2);
-                        const uint64_t bd = make_smem_desc(b0 + stage * B_BYTES + kb * 32, 16, 1024, 2);
-                        tc_mma_nvfp4_pair(tmem_base, ad, bd, idesc, sfa_t + kb * 4, sfb_t + kb * 8, (ks | kb) != 0);
+                        for (int kb = 0; kb < KB; ++kb)
+                            tc_mma_nvfp4_pair(tmem_base, make_smem_desc(a_s + kb * 32, 16, 1024, 2),
+                                              make_smem_desc(b_s + kb * 32, 16, 1024, 2), idesc, sfa_t + kb * 4,
+                                              sfb_t + kb * 8, (ks | kb) != 0);
+                        tc_commit_pair_multicast(&empty[stage], 0x3);
                     }
-                    tc_commit_pair_multicast(&empty[stage], 0x3);
+                    __syncwarp();
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -216,12 +223,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit_pair_multicast(acc_full, 0x3);
+                if (elect_one())
+                    tc_commit_pair_multicast(acc_full, 0x3);
+                __syncwarp();
                 acc_phase ^= 1u;
             }
-            tc_commit_pair(final_bar);
+            if (elect_one())
+                tc_commit_pair(final_bar);
+            __syncwarp();
+            // Wait for the last MMAs even when another role gave up (abort set):
+            // the tensor memory is released only after they are done.
             volatile int no_abort = 0;
-            if (!mbar_wait_bounded(final_bar, 0, &no_abort, DRAIN_TIMEOUT_NS))
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(final_bar, 0, &no_abort, DRAIN_TIMEOUT_NS)))
                 *abort_flag = 1;
         }
     } else {

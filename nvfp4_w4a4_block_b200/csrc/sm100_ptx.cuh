@@ -24,6 +24,20 @@ __device__ __forceinline__ uint64_t global_timer_ns()
     return t;
 }
 
+// One lane of a converged warp (the lowest active one) gets true.  Issuing
+// single-thread instructions (TMA, tcgen05) from an elected lane of a whole
+// warp keeps their operands warp-uniform, unlike a lane-divergent branch.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xFFFFFFFF;\n\t"
+        "selp.b32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
