@@ -501,7 +501,50 @@ def secondary_workloads(nv, W, peaks, fp4_peak):
         static_ms=round(ts, 4), static_gbs=round(b_static / (ts * 1e-3) / 1e9, 1),
         static_frac_hbm=round(b_static / (ts * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         bytes_dynamic=int(b_dyn), bytes_static=int(b_static))
-    del x, q, sf, flush_buf
+    del x, q, sf
+    torch.cuda.empty_cache()
+    out.update(conversion_workloads(nv, W, peaks, flush))
+    del flush_buf
+    torch.cuda.empty_cache()
+    return out
+
+
+def conversion_workloads(nv, W, peaks, flush):
+    """Expansion of the decode weights to bf16, checkpoint import of their block
+    scales, and harmonization of the fused q/k/v/gate scales (GB/s vs HBM, each
+    rep timed alone after an L2 flush)."""
+    import torch
+    out = {}
+
+    def entry(ms, nbytes):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return dict(ms=round(ms, 4), gbs=round(gbs, 1), frac_hbm=round(gbs / peaks["hbm_gbs"], 4), bytes=int(nbytes))
+
+    wl = W.DECODE
+    n, k, off = wl.n, wl.k, wl.seg_offsets
+    w = gen_device((n, k), "normal", 51, sigma=0.02)
+    w[off[1]:] *= 2.75
+    pw = nv.pack_weight(w, off)
+    del w
+    y = torch.empty((n, k), dtype=torch.bfloat16, device="cuda")
+    t = statistics.median(time_reps(lambda: nv.dequantize(pw.q, pw.sf, k, pw.gscale, off, out=y), 10, 3, flush))
+    out[f"dequantize_{n}x{k}"] = entry(t, n * k * (0.5 + 1 / 16 + 2))
+    del y
+    lin = torch.randint(0, 0x7F, (n, k // 16), dtype=torch.uint8, device="cuda")
+    sfo = torch.empty_like(pw.sf)
+    t = statistics.median(time_reps(lambda: nv.import_weight_scales(lin, n, k, out=sfo), 10, 3, flush))
+    out[f"import_scales_{n}x{k}"] = entry(t, n * k // 16 + sfo.numel())
+    del lin, sfo, pw
+    wl = W.FUSED_QKVG
+    n, k, off = wl.n, wl.k, wl.seg_offsets
+    w = gen_device((n, k), "normal", 52)
+    for i in range(len(off) - 1):
+        w[off[i]:off[i + 1]] *= float(wl.seg_sigma[i])
+    pw = nv.pack_weight(w, off)
+    del w
+    t = statistics.median(time_reps(lambda: nv.harmonize_scales(pw), 10, 3, flush))
+    out[f"harmonize_{n}x{k}"] = entry(t, 2 * pw.sf.numel())
+    del pw
     torch.cuda.empty_cache()
     return out
 
@@ -633,6 +676,29 @@ def _prof_decode_call(m, launches):
     assert nv.get_device_error() == nv.OK
 
 
+def _prof_convert(kind, launches):
+    import torch
+
+    import nvfp4_w4a4_block_b200 as nv
+    n, k, off = 34816, 5120, [0, 17408, 34816]
+    w = gen_device((n, k), "normal", 5, sigma=0.02)
+    pw = nv.pack_weight(w, off)
+    del w
+    y = torch.empty((n, k), dtype=torch.bfloat16, device="cuda") if kind == "dequantize" else None
+    lin = torch.randint(0, 0x7F, (n, k // 16), dtype=torch.uint8, device="cuda") if kind == "import" else None
+    sfo = torch.empty_like(pw.sf)
+    torch.cuda.synchronize()
+    for _ in range(launches):
+        if kind == "dequantize":
+            nv.dequantize(pw.q, pw.sf, k, pw.gscale, off, out=y)
+        elif kind == "import":
+            nv.import_weight_scales(lin, n, k, out=sfo)
+        else:
+            nv.harmonize_scales(pw)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+
+
 PROFILE_CASES = {
     "gemm_decode_m32": lambda L: _prof_gemm(32, 34816, 5120, [0, 17408, 34816], L),
     "gemm_prefill_8192x17408x5120": lambda L: _prof_gemm(8192, 17408, 5120, [0, 17408], L, "student_t3"),
@@ -640,6 +706,9 @@ PROFILE_CASES = {
     "quantize_32768x17408_static": lambda L: _prof_quantize(32768, 17408, L, True),
     "quantize_32768x17408_dynamic": lambda L: _prof_quantize(32768, 17408, L, False),
     "decode_call_m32": lambda L: _prof_decode_call(32, L),
+    "dequantize_34816x5120": lambda L: _prof_convert("dequantize", L),
+    "import_scales_34816x5120": lambda L: _prof_convert("import", L),
+    "harmonize_34816x5120": lambda L: _prof_convert("harmonize", L),
 }
 
 

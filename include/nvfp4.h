@@ -52,7 +52,7 @@
  *
  * Shape limits: K % 64 == 0, N % 8 == 0, M >= 0 (M == 0 is a no-op),
  * 1 <= nseg <= NVFP4_MAX_SEGMENTS, segment offsets strictly increasing from 0
- * to N (each a multiple of 8).
+ * to the segmented extent (N, or the row count), interior offsets multiples of 8.
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_
@@ -186,6 +186,65 @@ nvfp4_status nvfp4_linear_fused_noalloc(const void *x, int64_t m, int64_t k, int
                                         const uint8_t *qw, const uint8_t *sfw, int64_t n,
                                         const int64_t *seg_offsets, const float *seg_gscales, int nseg,
                                         void *y, int64_t ldy, unsigned flags, nvfp4_stream_t stream);
+
+/* Expansion of packed NVFP4 rows to bf16 (the "expand to BF16" step of the
+ * Gemma-4-31B-IT-NVFP4-FP8attn-text model card, §Limitations; it is the
+ * inverse of the encoding of "Why Gated DeltaNet Survives 4-Bit Quantization",
+ * §2 "NVFP4").  Element (r, j) is
+ *     y[r, j] = bf16( value(code[r, j]) * value(sf[r, j/16]) * s[segment(r)] )
+ * where the product is exact and is rounded once to the nearest bf16, ties to
+ * the even significand.
+ * q            device [rows, k/2] packed codes (16-byte aligned).
+ * sf           device block scales in the tensor-core layout (nvfp4_sf_bytes(rows, k)).
+ * seg_offsets  host int64[nseg+1] row segments (NULL with nseg == 1).
+ * seg_gscales  device float[nseg] global scale of each segment; they must be
+ *              finite (a non-finite scale gives unspecified values).
+ * y            device bf16 [rows, k] with row stride ldy elements (16-byte aligned rows).
+ * K % 64 == 0; any row count (rows == 0 is a no-op).  Needs no workspace. */
+nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t k,
+                              const int64_t *seg_offsets, const float *seg_gscales, int nseg,
+                              void *y, int64_t ldy, nvfp4_stream_t stream);
+
+/* Checkpoint import of block scales.  NVFP4 checkpoints store, per linear
+ * layer, the packed codes (uint8 [n, k/2], the same nibble order as Q above,
+ * so they are used as they are), the E4M3 block scales as a plain row-major
+ * matrix [n, k/16] (one byte per 16-element block) and the FP32 global scale,
+ * which is the dequantization multiplier s of this library ("Why Gated
+ * DeltaNet Survives 4-Bit Quantization", §3 "Checkpoints"; model card
+ * §Verification: max(block scale) x global x 6 = absmax).  This call
+ * rewrites the row-major block-scale matrix into the tensor-core layout.
+ * sf_linear  device [n, k/16] bytes with row stride ld_sf bytes (ld_sf >= k/16,
+ *            ld_sf % 4 == 0, base 4-byte aligned).
+ * sf_out     device nvfp4_sf_bytes(n, k) bytes, 16-byte aligned, not
+ *            overlapping sf_linear; pad bytes are written as 0.
+ * n == 0 is a no-op.  Needs no workspace. */
+nvfp4_status nvfp4_import_weight_scales(const uint8_t *sf_linear, int64_t n, int64_t k, int64_t ld_sf,
+                                        uint8_t *sf_out, nvfp4_stream_t stream);
+
+/* Harmonization of a fused group: the checkpoint-side repair of "Why Gated
+ * DeltaNet Survives 4-Bit Quantization", §6 "Per-module calibration vs.
+ * fused-GEMM scaling".  The modules concatenated along N keep their packed
+ * codes; the group gets one global scale s_shared = max_i seg_gscales[i], and
+ * every block scale of module i becomes
+ *     E4M3_rne_satfinite( value(sb) * (seg_gscales[i] / s_shared) )
+ * with the ratio and the product in fp32.  Every ratio is <= 1, so no folded
+ * scale passes 448; the re-rounding error is at most half an E4M3 ulp (2^-4
+ * relative in the normal range; the paper reports <= 6.2%).  Afterwards the
+ * weight can be served by a single-scale GEMM (nvfp4_linear with *w_gscale =
+ * s_shared).
+ * sf_in, sf_out   device block scales in the tensor-core layout
+ *                 (nvfp4_sf_bytes(n, k)), 16-byte aligned; sf_out may equal
+ *                 sf_in (in place) but must not partially overlap it.
+ * seg_offsets     host int64[nseg+1] (NULL with nseg == 1).
+ * seg_gscales     device float[nseg].
+ * shared_gscale_out device float, receives s_shared.
+ * A negative or non-finite module scale leaves the scales unchanged, writes
+ * NaN to *shared_gscale_out and records NVFP4_ERR_NONFINITE in the device error
+ * word.  An all-zero group is left unchanged (s_shared = 0).  Pad rows are
+ * copied unchanged.  Needs no workspace. */
+nvfp4_status nvfp4_harmonize_scales(const uint8_t *sf_in, uint8_t *sf_out, int64_t n, int64_t k,
+                                    const int64_t *seg_offsets, const float *seg_gscales, int nseg,
+                                    float *shared_gscale_out, nvfp4_stream_t stream);
 
 /* Synchronizes `stream`, then returns and clears the current device's error
  * word: NVFP4_ERR_NONFINITE, NVFP4_ERR_TIMEOUT, or NVFP4_OK. */

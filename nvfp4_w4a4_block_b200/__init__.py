@@ -12,6 +12,9 @@ Entry points mirror the C names:
   gemm(qx, sfx, s_x, pw, ...)             -> y
   linear(x, pw, act_gscale=None, ...)     -> y      (one module)
   linear_fused(x, pw, act_gscale=None...) -> y      (modules fused along N)
+  dequantize(q, sf, k, gscale, ...)       -> y bf16 (expansion of packed rows)
+  import_weight_scales(sf_linear, n, k)   -> sf     (checkpoint scales -> tensor-core layout)
+  harmonize_scales(pw)                    -> PackedWeight with one shared global scale
 """
 from __future__ import annotations
 
@@ -42,7 +45,8 @@ MAX_SEGMENTS = 8
 
 EXPORTED = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize_act",
             "nvfp4_pack_weight", "nvfp4_gemm", "nvfp4_linear", "nvfp4_linear_fused", "nvfp4_get_device_error",
-            "nvfp4_set_wait_timeout_ns", "nvfp4_version", "nvfp4_linear_fused_noalloc")
+            "nvfp4_set_wait_timeout_ns", "nvfp4_version", "nvfp4_linear_fused_noalloc", "nvfp4_dequantize",
+            "nvfp4_import_weight_scales", "nvfp4_harmonize_scales")
 
 
 class NVFP4Error(RuntimeError):
@@ -86,6 +90,12 @@ def lib() -> ctypes.CDLL:
                 L.nvfp4_linear_fused_noalloc.argtypes = [vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, ci, vp, i64,
                                                          u32, vp]
                 L.nvfp4_linear_fused_noalloc.restype = ci
+                L.nvfp4_dequantize.argtypes = [vp, vp, i64, i64, vp, vp, ci, vp, i64, vp]
+                L.nvfp4_dequantize.restype = ci
+                L.nvfp4_import_weight_scales.argtypes = [vp, i64, i64, i64, vp, vp]
+                L.nvfp4_import_weight_scales.restype = ci
+                L.nvfp4_harmonize_scales.argtypes = [vp, vp, i64, i64, vp, vp, ci, vp, vp]
+                L.nvfp4_harmonize_scales.restype = ci
                 _lib = L
     return _lib
 
@@ -276,3 +286,42 @@ def linear_fused_noalloc(x, pw: PackedWeight, act_gscale=None, out=None, flags: 
                                           _stream(stream))
     _check(st, "nvfp4_linear_fused_noalloc")
     return y
+
+
+def dequantize(q, sf, k: int, gscale, seg_offsets: Optional[Sequence[int]] = None, out=None, stream=None):
+    """Expand packed rows to bf16: value(code) * value(block scale) * s, rounded once.
+    q: [rows, k/2] uint8; sf: physical scales; gscale: device float32 [nseg]."""
+    torch = _torch()
+    rows = q.shape[0]
+    y = torch.empty((rows, k), dtype=torch.bfloat16, device=q.device) if out is None else out
+    offs = list(seg_offsets) if seg_offsets is not None else [0, rows]
+    arr, nseg = _seg_array(offs)
+    st = lib().nvfp4_dequantize(_ptr(q), _ptr(sf), rows, k, arr, _ptr(gscale), nseg, _ptr(y), y.stride(0),
+                                _stream(stream))
+    _check(st, "nvfp4_dequantize")
+    return y
+
+
+def import_weight_scales(sf_linear, n: int, k: int, out=None, stream=None):
+    """Checkpoint block scales [n, k/16] (uint8 E4M3, row-major, row stride
+    sf_linear.stride(0)) -> the tensor-core layout used by the GEMM."""
+    torch = _torch()
+    sf = torch.empty(sf_bytes(n, k), dtype=torch.uint8, device=sf_linear.device) if out is None else out
+    st = lib().nvfp4_import_weight_scales(_ptr(sf_linear), n, k, sf_linear.stride(0), _ptr(sf), _stream(stream))
+    _check(st, "nvfp4_import_weight_scales")
+    return sf
+
+
+def harmonize_scales(pw: PackedWeight, in_place: bool = False, stream=None) -> PackedWeight:
+    """Fold the per-module global scales of a fused weight into its block scales
+    so that one shared scale (the largest) serves the whole GEMM.  Returns a
+    single-segment PackedWeight sharing pw's codes."""
+    torch = _torch()
+    sf = pw.sf if in_place else torch.empty_like(pw.sf)
+    shared = torch.empty(1, dtype=torch.float32, device=pw.sf.device)
+    arr, nseg = _seg_array(pw.seg_offsets)
+    st = lib().nvfp4_harmonize_scales(_ptr(pw.sf), _ptr(sf), pw.n, pw.k, arr, _ptr(pw.gscale), nseg, _ptr(shared),
+                                      _stream(stream))
+    _check(st, "nvfp4_harmonize_scales")
+    return PackedWeight(pw.q, sf, shared, pw.n, pw.k, [0, pw.n])
+

@@ -1,0 +1,290 @@
+// convert.cuh -- kernels that rewrite packed NVFP4 tensors rather than multiply
+// them: expansion to bf16, checkpoint import of linear-layout block scales, and
+// harmonization of a fused group's global scales.  All three are HBM-bound
+// streams over the packed bytes.
+//
+//   * Expansion ("Gemma-4-31B-IT-NVFP4-FP8attn-text" model card, §Limitations:
+//     a packed checkpoint is expanded to BF16 to load it elsewhere).  Element j
+//     of row r becomes the bf16 nearest to value(code) * value(block scale) * s,
+//     rounded once (ties to even).  Per 16-element block only eight magnitudes
+//     occur; they are rounded exactly once per block into an 8-entry table, and
+//     each element is a table look-up (byte permutes) plus its sign bit.
+//   * Import ("Why Gated DeltaNet Survives 4-Bit Quantization", §3 "Checkpoints";
+//     model card §Verification: packed codes, per-block E4M3 weight_scale and the
+//     FP32 weight_scale_2): a [rows, K/16] block-scale matrix is scattered into
+//     the tensor-core atom layout; the packed codes are already in the layout the
+//     GEMM reads.
+//   * Harmonization (same paper, §6 "Per-module calibration vs. fused-GEMM
+//     scaling", the checkpoint-side repair): the fused group takes the largest of
+//     its modules' global scales and every block scale of module i is re-rounded
+//     to E4M3 after multiplying it by s_i / s_shared (both in fp32).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "quantize.cuh"
+
+namespace nvfp4 {
+namespace convert {
+
+constexpr int kThreads = 256;
+
+// ------------------------------------------------------------------ exact bf16 rounding
+
+// bf16 bits of the value p * s rounded once to nearest (ties to even), for p with
+// at most 24 significant bits and s any fp32.  The fp32 product hi is exact up to
+// its rounding error lo = fma(p, s, -hi); hi rounds to the same bf16 as p * s
+// unless hi sits exactly on a bf16 midpoint, where the sign of lo decides.  Tiny
+// products (below 2^-120, where lo may not be representable) go through fp64,
+// where the product is exact.
+__device__ __forceinline__ uint32_t bf16_bits_of_product(float p, float s)
+{
+    const float hi = __fmul_rn(p, s);
+    const uint32_t u = __float_as_uint(hi);
+    const uint32_t mag = u & 0x7FFFFFFFu;
+    if (mag >= 0x7F800000u)                           // inf (or NaN from inf * 0)
+        return (u >> 16) | (mag > 0x7F800000u ? 0x40u : 0u);
+    if (mag == 0u)
+        return u >> 16;
+    if (mag < 0x03800000u) {                          // |hi| < 2^-120
+        const __nv_bfloat16 b = __double2bfloat16(static_cast<double>(p) * static_cast<double>(s));
+        return static_cast<uint32_t>(__bfloat16_as_ushort(b));
+    }
+    uint32_t r = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+    if ((u & 0xFFFFu) == 0x8000u) {
+        const float lo = __fmaf_rn(p, s, -hi);
+        if (lo != 0.0f)
+            r = (u >> 16) + (((lo > 0.0f) == (hi > 0.0f)) ? 1u : 0u);
+    }
+    return r & 0xFFFFu;
+}
+
+// E2M1 magnitude code (0..7) -> value (0, 0.5, 1, 1.5, 2, 3, 4, 6).
+__device__ __forceinline__ float e2m1_magnitude(uint32_t m)
+{
+    if (m < 2u)
+        return 0.5f * static_cast<float>(m);
+    return __uint_as_float(((126u + (m >> 1)) << 23) | ((m & 1u) << 22));
+}
+
+// The eight bf16 magnitudes of one block, split into a low-byte table (lo0: entries
+// 0..3, lo1: 4..7) and a high-byte table, for byte-permute look-ups.  The E2M1
+// magnitudes are 1 and 1.5 times powers of two, and rounding commutes with a
+// power-of-two scaling while both values stay normal; so only value(sb)*s and
+// 1.5*value(sb)*s are rounded, and the rest are exponent shifts of those two.
+// Outside that range every entry is rounded on its own.
+struct BlockTable {
+    uint32_t lo0, lo1, hi0, hi1;
+};
+
+__device__ __forceinline__ BlockTable block_table(float sd, float s)
+{
+    uint32_t e[8];
+    e[0] = 0u;
+    const uint32_t c1 = bf16_bits_of_product(sd, s);
+    const uint32_t c15 = bf16_bits_of_product(1.5f * sd, s);       // exact: sd has 4 significant bits
+    const uint32_t x1 = (c1 >> 7) & 0xFFu, x15 = (c15 >> 7) & 0xFFu;
+    if (x1 >= 3u && x1 <= 252u && x15 >= 2u && x15 <= 252u) {
+        e[1] = c1 - 0x80u;       // 0.5
+        e[2] = c1;               // 1
+        e[3] = c15;              // 1.5
+        e[4] = c1 + 0x80u;       // 2
+        e[5] = c15 + 0x80u;      // 3
+        e[6] = c1 + 0x100u;      // 4
+        e[7] = c15 + 0x100u;     // 6
+    } else {
+#pragma unroll
+        for (int m = 1; m < 8; ++m)
+            e[m] = bf16_bits_of_product(e2m1_magnitude(m) * sd, s);   // e2m1 * e4m3 is exact in fp32
+    }
+    BlockTable t;
+    t.lo0 = (e[0] & 0xFFu) | ((e[1] & 0xFFu) << 8) | ((e[2] & 0xFFu) << 16) | ((e[3] & 0xFFu) << 24);
+    t.lo1 = (e[4] & 0xFFu) | ((e[5] & 0xFFu) << 8) | ((e[6] & 0xFFu) << 16) | ((e[7] & 0xFFu) << 24);
+    t.hi0 = (e[0] >> 8) | ((e[1] >> 8) << 8) | ((e[2] >> 8) << 16) | ((e[3] >> 8) << 24);
+    t.hi1 = (e[4] >> 8) | ((e[5] >> 8) << 8) | ((e[6] >> 8) << 16) | ((e[7] >> 8) << 24);
+    return t;
+}
+
+// Four codes (nibbles 0..3 of `w`, element order) -> two words of bf16 pairs.
+__device__ __forceinline__ void expand4(const BlockTable &t, uint32_t w, uint32_t &out0, uint32_t &out1)
+{
+    const uint32_t sel = w & 0x7777u;                          // magnitude indices
+    const uint32_t lo = __byte_perm(t.lo0, t.lo1, sel);        // low bytes of elements 0..3
+    const uint32_t hi = __byte_perm(t.hi0, t.hi1, sel);        // high bytes of elements 0..3
+    // sign bits: code bit 3 -> bf16 bit 15 of the element's half-word
+    const uint32_t s01 = ((w & 0x8u) << 12) | ((w & 0x80u) << 24);
+    const uint32_t s23 = ((w & 0x800u) << 4) | ((w & 0x8000u) << 16);
+    out0 = __byte_perm(lo, hi, 0x5140u) | s01;
+    out1 = __byte_perm(lo, hi, 0x7362u) | s23;
+}
+
+// ------------------------------------------------------------------ expansion
+
+struct ExpandParams {
+    const uint8_t *q;          // [rows, k/2]
+    const uint8_t *sf;         // physical scales
+    uint16_t *y;               // bf16 [rows, ldy]
+    int64_t rows, k, ldy;
+    int64_t row_tiles, col_tiles;   // 128-row x 64-column tiles (one scale atom each)
+    int nseg;
+    int64_t seg_end[kMaxSeg];
+    const float *gscale;       // [nseg] device
+};
+
+// One tile = 128 rows x 64 elements = one 512-byte scale atom.  Thread t owns
+// 32 elements (two blocks) of row t/2: 16 bytes of codes in, 64 bytes out.
+__global__ void __launch_bounds__(kThreads) expand_kernel(ExpandParams p)
+{
+    __shared__ float s_scale[kMaxSeg];
+    if (threadIdx.x < kMaxSeg)
+        s_scale[threadIdx.x] = threadIdx.x < static_cast<unsigned>(p.nseg) ? p.gscale[threadIdx.x] : 0.0f;
+    __syncthreads();
+    const int r_in = threadIdx.x >> 1;          // row inside the tile
+    const int half = threadIdx.x & 1;           // which 32 elements of the 64
+    const int64_t tiles = p.row_tiles * p.col_tiles;
+    const int64_t kh = p.k >> 1;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t rt = t / p.col_tiles, ct = t - rt * p.col_tiles;
+        const int64_t row = rt * 128 + r_in;
+        if (row >= p.rows)
+            continue;
+        const uint4 codes = __ldg(reinterpret_cast<const uint4 *>(p.q + row * kh + ct * 32 + half * 16));
+        const uint8_t *atom = p.sf + (rt * p.col_tiles + ct) * 512 + (r_in & 31) * 16 + (r_in >> 5) * 4 + half * 2;
+        const uint32_t sf2 = __ldg(reinterpret_cast<const uint16_t *>(atom));
+        int seg = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxSeg - 1; ++i)
+            seg += (i + 1 < p.nseg && row >= p.seg_end[i]) ? 1 : 0;
+        const float s = s_scale[seg];
+        const BlockTable t0 = block_table(e4m3_to_f32(sf2 & 0xFFu), s);
+        const BlockTable t1 = block_table(e4m3_to_f32(sf2 >> 8), s);
+        uint4 o0, o1, o2, o3;
+        expand4(t0, codes.x, o0.x, o0.y);
+        expand4(t0, codes.x >> 16, o0.z, o0.w);
+        expand4(t0, codes.y, o1.x, o1.y);
+        expand4(t0, codes.y >> 16, o1.z, o1.w);
+        expand4(t1, codes.z, o2.x, o2.y);
+        expand4(t1, codes.z >> 16, o2.z, o2.w);
+        expand4(t1, codes.w, o3.x, o3.y);
+        expand4(t1, codes.w >> 16, o3.z, o3.w);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.y + row * p.ldy + ct * 64 + half * 32);
+        dst[0] = o0;
+        dst[1] = o1;
+        dst[2] = o2;
+        dst[3] = o3;
+    }
+}
+
+// ------------------------------------------------------------------ checkpoint import
+
+struct ImportParams {
+    const uint8_t *lin;        // [rows, k/16] bytes, row stride ld (bytes, multiple of 4)
+    uint8_t *sf;               // physical scales
+    int64_t rows, ld;
+    int64_t row_tiles, atoms_k;     // tiles are 128 rows x 16 atoms (64 scale columns)
+    int64_t col_groups;             // ceil(atoms_k / 16)
+};
+
+// One tile = 128 rows x 64 scale columns: rows are read as 4-byte words (one
+// atom's four columns) and the 16 atoms leave as one contiguous 8 KB run.
+__global__ void __launch_bounds__(kThreads) import_scales_kernel(ImportParams p)
+{
+    const int64_t tiles = p.row_tiles * p.col_groups;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t rt = t / p.col_groups, cg = t - rt * p.col_groups;
+        const int64_t a0 = cg * 16;
+        const int natoms = static_cast<int>(p.atoms_k - a0 < 16 ? p.atoms_k - a0 : 16);
+        // 16 atoms x 32 words of 16 bytes; thread handles word w of atom a.
+        for (int i = threadIdx.x; i < natoms * 32; i += blockDim.x) {
+            const int a = i >> 5, w = i & 31;     // atom, and row-in-quarter (r % 32)
+            uint32_t v[4];
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+                const int64_t row = rt * 128 + qd * 32 + w;
+                v[qd] = row < p.rows
+                            ? __ldg(reinterpret_cast<const uint32_t *>(p.lin + row * p.ld + (a0 + a) * 4))
+                            : 0u;
+            }
+            *reinterpret_cast<uint4 *>(p.sf + (rt * p.atoms_k + a0 + a) * 512 + w * 16) =
+                make_uint4(v[0], v[1], v[2], v[3]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ harmonization
+
+struct HarmonizeParams {
+    const uint8_t *sf_in;
+    uint8_t *sf_out;           // may alias sf_in
+    int64_t rows, atoms_k;     // atoms along K per 128-row block
+    int64_t units;             // 16-byte words of the physical buffer
+    int nseg;
+    int64_t seg_end[kMaxSeg];
+    const float *gscale;       // [nseg] device
+    float *shared_out;         // 1 float, device
+};
+
+// Thread handles one 16-byte word of an atom: rows 32j + (word index) of the
+// atom's 128-row block, j = 0..3, four scale columns each.  Each CTA derives the
+// shared scale and the per-module ratios itself from the device scales.
+__global__ void __launch_bounds__(kThreads) harmonize_kernel(HarmonizeParams p)
+{
+    __shared__ float s_ratio[kMaxSeg];
+    __shared__ int s_state;                    // 0 fold, 1 copy unchanged (all zero), 2 bad scale
+    if (threadIdx.x == 0) {
+        float shared = 0.0f;
+        int bad = 0;
+        for (int i = 0; i < p.nseg; ++i) {
+            const float g = p.gscale[i];
+            if (!(g >= 0.0f) || isinf(g))
+                bad = 1;
+            else
+                shared = fmaxf(shared, g);
+        }
+        s_state = bad ? 2 : (shared == 0.0f ? 1 : 0);
+        for (int i = 0; i < kMaxSeg; ++i)
+            s_ratio[i] = (!bad && shared != 0.0f && i < p.nseg) ? __fdiv_rn(p.gscale[i], shared) : 1.0f;
+        if (blockIdx.x == 0) {
+            *p.shared_out = bad ? __int_as_float(0x7FC00000) : shared;
+            if (bad)
+                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
+        }
+    }
+    __syncthreads();
+    const int state = s_state;
+    if (state == 2)
+        return;                                // leave the scales as they are
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < p.units; u += nthreads) {
+        uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.sf_in) + u);
+        if (state == 0) {
+            const int64_t rb = (u >> 5) / p.atoms_k;
+            const int w = static_cast<int>(u & 31);
+            uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t row = rb * 128 + j * 32 + w;
+                if (row >= p.rows)
+                    continue;                  // pad rows stay as they are
+                int seg = 0;
+#pragma unroll
+                for (int i = 0; i < kMaxSeg - 1; ++i)
+                    seg += (i + 1 < p.nseg && row >= p.seg_end[i]) ? 1 : 0;
+                const float ratio = s_ratio[seg];
+                uint32_t out = 0;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const float folded = __fmul_rn(e4m3_to_f32((words[j] >> (8 * b)) & 0xFFu), ratio);
+                    out |= f32_to_e4m3(folded) << (8 * b);
+                }
+                words[j] = out;
+            }
+            v = make_uint4(words[0], words[1], words[2], words[3]);
+        }
+        reinterpret_cast<uint4 *>(p.sf_out)[u] = v;
+    }
+}
+
+}  // namespace convert
+}  // namespace nvfp4

@@ -17,7 +17,7 @@
 //     the activation quantizer that precedes it is still running, then loads the
 //     activation stages.
 //
-// Roles: warp 0 producer (TMA + bulk copies), warp 1 MMA issuer (one thread),
+// Roles: warp 0 producer (TMA + bulk copies), warp 1 MMA issuer (one elected lane),
 // warps 2..5 epilogue (tcgen05.ld of the 128 x T accumulator, x alpha(n), bf16
 // stores of Y[t, n] -- 32 consecutive n per warp per token).
 #pragma once
@@ -121,96 +121,109 @@ __global__ void __launch_bounds__(THREADS, 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            const int pre = min(C::STAGES, p.k_stages);
-            // Weight stages first: they do not depend on the preceding kernel.
-            for (int ks = 0; ks < pre; ++ks) {
-                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+        // The whole warp walks the schedule (operands stay warp-uniform); one
+        // elected lane issues the copies.
+        const int pre = min(C::STAGES, p.k_stages);
+        // Weight stages first: they do not depend on the preceding kernel.
+        for (int ks = 0; ks < pre; ++ks) {
+            const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+            const uint8_t *sfw_src = p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512;
+            if (elect_one()) {
                 mbar_arrive_expect_tx(&full[ks], A_BYTES + C::B_BYTES + 2 * nkb * 512);
                 tma_load_2d(smem + C::OFF_A + ks * A_BYTES, &tm_w, ks * (BK / 2), w0, &full[ks]);
-                bulk_load(smem + C::OFF_SFA + ks * SF_BYTES,
-                          p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512, nkb * 512,
+                bulk_load(smem + C::OFF_SFA + ks * SF_BYTES, sfw_src, nkb * 512, &full[ks]);
+            }
+            __syncwarp();
+        }
+        pdl_wait_prerequisites();                // activation codes/scales are now written
+        for (int ks = 0; ks < pre; ++ks) {
+            const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+            if (elect_one()) {
+                tma_load_2d(smem + C::OFF_B + ks * C::B_BYTES, &tm_x, ks * (BK / 2), 0, &full[ks]);
+                bulk_load(smem + C::OFF_SFB + ks * SF_BYTES, p.sfx + static_cast<int64_t>(ks * KB) * 512, nkb * 512,
                           &full[ks]);
             }
-            pdl_wait_prerequisites();            // activation codes/scales are now written
-            for (int ks = 0; ks < pre; ++ks) {
-                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
-                tma_load_2d(smem + C::OFF_B + ks * C::B_BYTES, &tm_x, ks * (BK / 2), 0, &full[ks]);
-                bulk_load(smem + C::OFF_SFB + ks * SF_BYTES, p.sfx + static_cast<int64_t>(ks * KB) * 512,
-                          nkb * 512, &full[ks]);
-            }
-            int stage = pre % C::STAGES;
-            uint32_t phase = (pre == C::STAGES) ? 1u : 0u;
-            int issued = pre;
-            for (int ks = pre; ks < p.k_stages; ++ks) {
-                if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns))
-                    break;
-                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+            __syncwarp();
+        }
+        int stage = pre % C::STAGES;
+        uint32_t phase = (pre == C::STAGES) ? 1u : 0u;
+        int issued = pre;
+        for (int ks = pre; ks < p.k_stages; ++ks) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)))
+                break;
+            const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+            const uint8_t *sfw_src = p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512;
+            if (elect_one()) {
                 mbar_arrive_expect_tx(&full[stage], A_BYTES + C::B_BYTES + 2 * nkb * 512);
                 tma_load_2d(smem + C::OFF_A + stage * A_BYTES, &tm_w, ks * (BK / 2), w0, &full[stage]);
-                bulk_load(smem + C::OFF_SFA + stage * SF_BYTES,
-                          p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512, nkb * 512,
-                          &full[stage]);
+                bulk_load(smem + C::OFF_SFA + stage * SF_BYTES, sfw_src, nkb * 512, &full[stage]);
                 tma_load_2d(smem + C::OFF_B + stage * C::B_BYTES, &tm_x, ks * (BK / 2), 0, &full[stage]);
                 bulk_load(smem + C::OFF_SFB + stage * SF_BYTES, p.sfx + static_cast<int64_t>(ks * KB) * 512,
                           nkb * 512, &full[stage]);
-                issued = ks + 1;
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
             }
-            // Every stage issued must have landed before the CTA exits: the last
-            // min(STAGES, issued) issues are the only ones possibly in flight.
-            for (int j = 0; j < min(C::STAGES, issued); ++j) {
-                const int ks = issued - 1 - j;
-                const int s = ks % C::STAGES;
-                const uint32_t ph = static_cast<uint32_t>((ks / C::STAGES) & 1);
-                volatile int no_abort = 0;
-                if (!mbar_wait_bounded(&full[s], ph, &no_abort, DRAIN_TIMEOUT_NS))
-                    *abort_flag = 1;
+            __syncwarp();
+            issued = ks + 1;
+            if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1u;
             }
+        }
+        // Every stage issued must have landed before the CTA exits: the last
+        // min(STAGES, issued) issues are the only ones possibly in flight.
+        for (int j = 0; j < min(C::STAGES, issued); ++j) {
+            const int ks = issued - 1 - j;
+            const int s = ks % C::STAGES;
+            const uint32_t ph = static_cast<uint32_t>((ks / C::STAGES) & 1);
+            volatile int no_abort = 0;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], ph, &no_abort, DRAIN_TIMEOUT_NS)))
+                *abort_flag = 1;
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc_nvfp4(BW, T);
-            const uint32_t sfa_t = tmem_base + C::TMEM_SFA;
-            const uint32_t sfb_t = tmem_base + C::TMEM_SFB;
-            const uint32_t a0 = smem_u32(smem + C::OFF_A), b0 = smem_u32(smem + C::OFF_B);
-            const uint32_t sfa0 = smem_u32(smem + C::OFF_SFA), sfb0 = smem_u32(smem + C::OFF_SFB);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int ks = 0; ks < p.k_stages; ++ks) {
-                if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+        // Warp-wide loop; the elected lane (lane 0 of the converged warp) issues
+        // every copy, MMA and commit, so its commits cover all its MMAs.
+        const uint32_t idesc = make_idesc_nvfp4(BW, T);
+        const uint32_t sfa_t = tmem_base + C::TMEM_SFA;
+        const uint32_t sfb_t = tmem_base + C::TMEM_SFB;
+        const uint32_t a0 = smem_u32(smem + C::OFF_A), b0 = smem_u32(smem + C::OFF_B);
+        const uint32_t sfa0 = smem_u32(smem + C::OFF_SFA), sfb0 = smem_u32(smem + C::OFF_SFB);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int ks = 0; ks < p.k_stages; ++ks) {
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns));
+            if (!ok)
+                break;
+            tc_fence_after();
+            const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
+            const uint32_t sfa_s = sfa0 + stage * SF_BYTES, sfb_s = sfb0 + stage * SF_BYTES;
+            const uint32_t a_s = a0 + stage * A_BYTES, b_s = b0 + stage * C::B_BYTES;
+            if (elect_one()) {
                 for (int kb = 0; kb < nkb; ++kb) {
-                    tc_cp_32x128b_warpx4(sfa_t + kb * 4, make_smem_desc(sfa0 + stage * SF_BYTES + kb * 512, 0, 128, 0));
-                    tc_cp_32x128b_warpx4(sfb_t + kb * 4, make_smem_desc(sfb0 + stage * SF_BYTES + kb * 512, 0, 128, 0));
+                    tc_cp_32x128b_warpx4(sfa_t + kb * 4, make_smem_desc(sfa_s + kb * 512, 0, 128, 0));
+                    tc_cp_32x128b_warpx4(sfb_t + kb * 4, make_smem_desc(sfb_s + kb * 512, 0, 128, 0));
                 }
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const uint64_t ad = make_smem_desc(a0 + stage * A_BYTES + kb * 32, 16, 1024, 2);
-                    const uint64_t bd = make_smem_desc(b0 + stage * C::B_BYTES + kb * 32, 16, 1024, 2);
-                    tc_mma_nvfp4(tmem_base, ad, bd, idesc, sfa_t + kb * 4, sfb_t + kb * 4, (ks | kb) != 0);
-                }
+                for (int kb = 0; kb < nkb; ++kb)
+                    tc_mma_nvfp4(tmem_base, make_smem_desc(a_s + kb * 32, 16, 1024, 2),
+                                 make_smem_desc(b_s + kb * 32, 16, 1024, 2), idesc, sfa_t + kb * 4, sfb_t + kb * 4,
+                                 (ks | kb) != 0);
                 tc_commit(&empty[stage]);
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
             }
+            __syncwarp();
+            if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (elect_one()) {
             if (ok)
                 tc_commit(acc_full);
             tc_commit(final_bar);
-            volatile int no_abort = 0;
-            if (!mbar_wait_bounded(final_bar, 0, &no_abort, DRAIN_TIMEOUT_NS))
-                *abort_flag = 1;
         }
+        __syncwarp();
+        volatile int no_abort = 0;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(final_bar, 0, &no_abort, DRAIN_TIMEOUT_NS)))
+            *abort_flag = 1;
     } else {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;

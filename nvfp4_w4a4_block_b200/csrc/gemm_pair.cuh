@@ -15,8 +15,10 @@
 //     stage barrier; the even CTA's tcgen05.commit releases the stage in both.
 //   * Eight epilogue warps per CTA drain the accumulator into registers (128
 //     columns each), hand the tensor memory back to the MMA issuer at once, and
-//     only then scale, convert and store -- the next tile's MMAs overlap the
-//     stores.
+//     only then scale and convert -- the next tile's MMAs overlap the rest of the
+//     epilogue.  bf16 results leave through a 32 KB shared-memory staging tile
+//     (two 128 x 64 sub-tiles, 128-byte swizzle: conflict-free 16-byte writes)
+//     in two rounds, one per 128-column half, each ending in two TMA stores.
 //   * Scale factors travel as 512-byte atoms through 3-D tensor maps; both CTAs
 //     load the full 256-row weight-scale block (no multicast of any kind).
 #pragma once
@@ -52,7 +54,9 @@ constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
 constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+constexpr int OFF_STG = OFF_SFB + STAGES * SFB_BYTES;   // bf16 output staging: 2 x [128 rows x 64 cols]
+constexpr int STG_SUB = 128 * 64 * 2;
+constexpr int OFF_BAR = OFF_STG + 2 * STG_SUB;
 constexpr int NUM_BARS = 2 * STAGES + 3;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_ALLOC = OFF_MISC + 64 + 1024;
@@ -75,21 +79,34 @@ struct Params {
     uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ float col_alpha(const Params &p, float sx, float swmax, int col)
+// Segment (module) of output column `col`.
+__device__ __forceinline__ int col_segment(const Params &p, int col)
 {
-    if (p.flags & FLAG_COLLAPSED)
-        return sx * swmax;
     int seg = 0;
 #pragma unroll
     for (int s = 0; s < 7; ++s)
         seg += (s + 1 < p.nseg && col >= p.seg_end[s]) ? 1 : 0;
-    return sx * p.s_w[seg];
+    return seg;
+}
+
+// Scales 32 accumulator columns starting at output column nc by their segment's
+// alpha (from the per-CTA table in shared memory).  Segment boundaries are
+// multiples of 8 columns, so one alpha serves each group of 8.
+__device__ __forceinline__ void scale32(const Params &p, const float *alpha, int nc, const uint32_t *r, float *v)
+{
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        const float a = alpha[col_segment(p, min(nc + 8 * g, p.n - 1))];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            v[8 * g + i] = __uint_as_float(r[8 * g + i]) * a;
+    }
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                            const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
-                           const Params p)
+                           const __grid_constant__ CUtensorMap tm_y, const Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -122,6 +139,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         prefetch_tensormap(&tm_b);
         prefetch_tensormap(&tm_sfa);
         prefetch_tensormap(&tm_sfb);
+        prefetch_tensormap(&tm_y);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -241,18 +259,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - 2;                        // 0..7
         const int quarter = warp & 3;                   // TMEM lanes this warp may read
-        const int col0 = (ew >> 2) * 128;               // this warp's 128 accumulator columns
+        const int half = ew >> 2;                       // this warp's 128 accumulator columns
+        const int col0 = half * 128;
+        const int row = quarter * 32 + lane;            // row inside this CTA's 128-row half tile
+        const bool issuer = (ew == 0 && lane == 0);     // issues the TMA stores
         pdl_wait_prerequisites();
-        const float sx = *p.s_x;
-        float swmax = p.s_w[0];
-        for (int s = 1; s < p.nseg; ++s)
-            swmax = fmaxf(swmax, p.s_w[s]);
+        // alpha of each segment: s_x * s_w[segment] (or s_x * max s_w for the
+        // collapsed negative control), computed once per CTA.
+        float *alpha = reinterpret_cast<float *>(smem + OFF_MISC + 16);
+        if (ew == 0 && lane == 0) {
+            const float sx = *p.s_x;
+            float swmax = p.s_w[0];
+            for (int s = 1; s < p.nseg; ++s)
+                swmax = fmaxf(swmax, p.s_w[s]);
+            for (int s = 0; s < p.nseg; ++s)
+                alpha[s] = (p.flags & FLAG_COLLAPSED) ? sx * swmax : sx * p.s_w[s];
+        }
+        bar_sync_named(2, 32 * EPI_WARPS);
         const bool f32_out = (p.flags & FLAG_F32_OUT) != 0;
         const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
+        uint8_t *stg = smem + OFF_STG;
         uint32_t acc_phase = 0;
         for (int tile = pair_id; tile < num_tiles; tile += npairs) {
             const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
-            if (!mbar_wait_bounded(acc_full, acc_phase, abort_flag, p.timeout_ns))
+            const bool ok = mbar_wait_bounded(acc_full, acc_phase, abort_flag, p.timeout_ns);
+            // All eight warps take the same decision (each reaches this barrier after
+            // its own bounded wait), so the named barriers below cannot strand one.
+            if (bar_red_or(1, 32 * EPI_WARPS, ok ? 0u : 1u))
                 break;
             tc_fence_after();
             uint32_t r[128];
@@ -269,39 +302,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 mbar_arrive_remote(acc_empty_leader);    // the accumulator may be overwritten now
             acc_phase ^= 1u;
 
-            const int m = mb * BM + static_cast<int>(rank) * 128 + quarter * 32 + lane;
-            if (m < p.m) {
+            const int m0 = mb * BM + static_cast<int>(rank) * 128;     // first row of this CTA's half tile
+            const int n0 = nb * BN;
+            if (!f32_out) {
+                // Scale and round this warp's 128 columns to packed bf16 pairs.
+                uint32_t pk[64];
 #pragma unroll
                 for (int c = 0; c < 128; c += 32) {
-                    const int nc = nb * BN + col0 + c;
-                    if (nc >= p.n)
-                        break;
-                    const float a_lo = col_alpha(p, sx, swmax, nc);
-                    const float a_hi = col_alpha(p, sx, swmax, min(nc + 31, p.n - 1));
                     float v[32];
+                    scale32(p, alpha, n0 + col0 + c, r + c, v);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        v[i] = __uint_as_float(r[c + i]) *
-                               (a_lo == a_hi ? a_lo : col_alpha(p, sx, swmax, min(nc + i, p.n - 1)));
-                    if (!f32_out) {
-                        __nv_bfloat16 *dst =
-                            reinterpret_cast<__nv_bfloat16 *>(p.y) + static_cast<int64_t>(m) * p.ldy + nc;
+                    for (int i = 0; i < 32; i += 2) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(v[i], v[i + 1]);
+                        pk[(c + i) >> 1] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                }
+                // Two rounds, one per 128-column half: the half's four warps write
+                // the staging tile, then one thread stores it.
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            if (nc + g * 8 < p.n) {
-                                __nv_bfloat162 h0 = __floats2bfloat162_rn(v[g * 8 + 0], v[g * 8 + 1]);
-                                __nv_bfloat162 h1 = __floats2bfloat162_rn(v[g * 8 + 2], v[g * 8 + 3]);
-                                __nv_bfloat162 h2 = __floats2bfloat162_rn(v[g * 8 + 4], v[g * 8 + 5]);
-                                __nv_bfloat162 h3 = __floats2bfloat162_rn(v[g * 8 + 6], v[g * 8 + 7]);
-                                uint4 o;
-                                o.x = *reinterpret_cast<uint32_t *>(&h0);
-                                o.y = *reinterpret_cast<uint32_t *>(&h1);
-                                o.z = *reinterpret_cast<uint32_t *>(&h2);
-                                o.w = *reinterpret_cast<uint32_t *>(&h3);
-                                *reinterpret_cast<uint4 *>(dst + g * 8) = o;
-                            }
+                for (int round = 0; round < 2; ++round) {
+                    // The previous stores must have finished reading the staging tile.
+                    if (issuer)
+                        bulk_wait_group_read0();
+                    bar_sync_named(2, 32 * EPI_WARPS);
+                    if (half == round) {
+#pragma unroll
+                        for (int chunk16 = 0; chunk16 < 16; ++chunk16) {       // 16 chunks of 8 columns
+                            const int sub = chunk16 >> 3, chunk = chunk16 & 7;
+                            uint8_t *base = stg + sub * STG_SUB + row * 128;
+                            *reinterpret_cast<uint4 *>(base + ((chunk ^ (row & 7)) << 4)) =
+                                make_uint4(pk[chunk16 * 4 + 0], pk[chunk16 * 4 + 1], pk[chunk16 * 4 + 2],
+                                           pk[chunk16 * 4 + 3]);
                         }
-                    } else {
+                        fence_async_shared();
+                    }
+                    bar_sync_named(2, 32 * EPI_WARPS);
+                    if (issuer && m0 < p.m) {
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub) {
+                            const int col = n0 + round * 128 + sub * 64;
+                            if (col < p.n)
+                                tma_store_2d(&tm_y, col, m0, stg + sub * STG_SUB);
+                        }
+                        bulk_commit_group();
+                    }
+                }
+            } else {
+                const int m = m0 + row;
+                if (m < p.m) {
+#pragma unroll
+                    for (int c = 0; c < 128; c += 32) {
+                        const int nc = n0 + col0 + c;
+                        if (nc >= p.n)
+                            break;
+                        float v[32];
+                        scale32(p, alpha, nc, r + c, v);
                         float *dst = reinterpret_cast<float *>(p.y) + static_cast<int64_t>(m) * p.ldy + nc;
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
@@ -316,6 +371,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
         }
+        if (issuer)
+            bulk_wait_group0();                         // every output store has completed
     }
 
     tc_fence_before();

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "nvfp4.h"
+#include "convert.cuh"
 #include "gemm_decode.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_sm100.cuh"
@@ -166,7 +167,7 @@ nvfp4_status read_segments(const int64_t *offsets, int nseg, int64_t total, int6
         if (offsets[i + 1] <= offsets[i])
             return NVFP4_ERR_INVALID_ARG;
     for (int i = 0; i < nseg; ++i) {
-        if (offsets[i + 1] % 8 != 0)
+        if (i + 1 < nseg && offsets[i + 1] % 8 != 0)      // interior boundaries; the total has its own limits
             return NVFP4_ERR_UNSUPPORTED_SHAPE;
         ends[i] = offsets[i + 1];
     }
@@ -302,13 +303,30 @@ nvfp4_status make_sf_map(CUtensorMap *map, const void *base, uint64_t atoms_k, u
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// bf16 output as a TMA store target: [m, n] with row stride ldy elements, boxes
+// of 64 columns x 128 rows with 128-byte swizzle (the epilogue's staging layout).
+nvfp4_status make_out_map(CUtensorMap *map, void *y, uint64_t m, uint64_t n, uint64_t ldy)
+{
+    cuuint64_t dims[2] = {n, m};
+    cuuint64_t strides[1] = {ldy * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
                          const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
                          const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms, bool pdl,
                          cudaStream_t stream)
 {
-    CUtensorMap ta, tb, tsa, tsb;
+    CUtensorMap ta, tb, tsa, tsb, ty;
+    memset(&ty, 0, sizeof ty);
     nvfp4_status st = make_map(&ta, qx, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(m), 128);
+    if (st == NVFP4_OK && !(flags & NVFP4_FLAG_F32_OUT))
+        st = make_out_map(&ty, y, static_cast<uint64_t>(m), static_cast<uint64_t>(n), static_cast<uint64_t>(ldy));
     if (st == NVFP4_OK)
         st = make_map(&tb, qw, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n), 128);
     if (st == NVFP4_OK)
@@ -337,7 +355,7 @@ nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
     return cuda_status(launch(pair::nvfp4_gemm_pair_kernel, static_cast<int>(2 * pairs), pair::THREADS,
-                              pair::SMEM_ALLOC, stream, pdl, ta, tb, tsa, tsb, p));
+                              pair::SMEM_ALLOC, stream, pdl, ta, tb, tsa, tsb, ty, p));
 }
 
 template <int T>
@@ -652,6 +670,129 @@ nvfp4_status nvfp4_linear_fused_noalloc(const void *x, int64_t m, int64_t k, int
     }
     return nvfp4_linear_fused(x, m, k, ldx, act_gscale, qw, sfw, n, seg_offsets, seg_gscales, nseg, y, ldy, flags,
                               ptr, NVFP4_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t k,
+                              const int64_t *seg_offsets, const float *seg_gscales, int nseg, void *y, int64_t ldy,
+                              nvfp4_stream_t stream)
+{
+    if (rows < 0 || k <= 0 || ldy < k)
+        return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0 || rows > (int64_t(1) << 31) || k > (int64_t(1) << 30))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0)
+        return seg_offsets == nullptr && nseg == 1 ? NVFP4_OK : NVFP4_ERR_INVALID_ARG;
+    int64_t ends[NVFP4_MAX_SEGMENTS];
+    nvfp4_status st = read_segments(seg_offsets, nseg, rows, ends);
+    if (st != NVFP4_OK)
+        return st;
+    if (q == nullptr || sf == nullptr || seg_gscales == nullptr || y == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(sf) || !aligned16(y) || (ldy * 2) % 16 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    if ((st = device_setup(&sms)) != NVFP4_OK)
+        return st;
+    convert::ExpandParams ep;
+    memset(&ep, 0, sizeof ep);
+    ep.q = q;
+    ep.sf = sf;
+    ep.y = static_cast<uint16_t *>(y);
+    ep.rows = rows;
+    ep.k = k;
+    ep.ldy = ldy;
+    ep.row_tiles = (rows + 127) / 128;
+    ep.col_tiles = k / 64;
+    ep.nseg = nseg;
+    for (int i = 0; i < nseg; ++i)
+        ep.seg_end[i] = ends[i];
+    ep.gscale = seg_gscales;
+    const int64_t tiles = ep.row_tiles * ep.col_tiles;
+    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    const int grid = static_cast<int>(tiles < cap ? tiles : cap);
+    return cuda_status(launch(convert::expand_kernel, grid, convert::kThreads, 0,
+                              reinterpret_cast<cudaStream_t>(stream), false, ep));
+}
+
+nvfp4_status nvfp4_import_weight_scales(const uint8_t *sf_linear, int64_t n, int64_t k, int64_t ld_sf,
+                                        uint8_t *sf_out, nvfp4_stream_t stream)
+{
+    if (n < 0 || k <= 0 || ld_sf < k / 16)
+        return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0 || n > (int64_t(1) << 31) || k > (int64_t(1) << 30))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (n == 0)
+        return NVFP4_OK;
+    if (sf_linear == nullptr || sf_out == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(sf_linear) & 3u) != 0 || ld_sf % 4 != 0 || !aligned16(sf_out))
+        return NVFP4_ERR_MISALIGNED;
+    const uintptr_t in0 = reinterpret_cast<uintptr_t>(sf_linear);
+    const uintptr_t in1 = in0 + static_cast<uintptr_t>((n - 1) * ld_sf + k / 16);
+    const uintptr_t out0 = reinterpret_cast<uintptr_t>(sf_out);
+    const uintptr_t out1 = out0 + nvfp4_sf_bytes(n, k);
+    if (in0 < out1 && out0 < in1)
+        return NVFP4_ERR_INVALID_ARG;        // the layouts differ, so no in-place import
+    int sms = 0;
+    nvfp4_status st = device_setup(&sms);
+    if (st != NVFP4_OK)
+        return st;
+    convert::ImportParams ip;
+    memset(&ip, 0, sizeof ip);
+    ip.lin = sf_linear;
+    ip.sf = sf_out;
+    ip.rows = n;
+    ip.ld = ld_sf;
+    ip.row_tiles = (n + 127) / 128;
+    ip.atoms_k = k / 64;
+    ip.col_groups = (ip.atoms_k + 15) / 16;
+    const int64_t tiles = ip.row_tiles * ip.col_groups;
+    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    const int grid = static_cast<int>(tiles < cap ? tiles : cap);
+    return cuda_status(launch(convert::import_scales_kernel, grid, convert::kThreads, 0,
+                              reinterpret_cast<cudaStream_t>(stream), false, ip));
+}
+
+nvfp4_status nvfp4_harmonize_scales(const uint8_t *sf_in, uint8_t *sf_out, int64_t n, int64_t k,
+                                    const int64_t *seg_offsets, const float *seg_gscales, int nseg,
+                                    float *shared_gscale_out, nvfp4_stream_t stream)
+{
+    if (n <= 0 || k <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0 || n > (int64_t(1) << 31) || k > (int64_t(1) << 30))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    int64_t ends[NVFP4_MAX_SEGMENTS];
+    nvfp4_status st = read_segments(seg_offsets, nseg, n, ends);
+    if (st != NVFP4_OK)
+        return st;
+    if (sf_in == nullptr || sf_out == nullptr || seg_gscales == nullptr || shared_gscale_out == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(sf_in) || !aligned16(sf_out))
+        return NVFP4_ERR_MISALIGNED;
+    const size_t bytes = nvfp4_sf_bytes(n, k);
+    const uintptr_t a = reinterpret_cast<uintptr_t>(sf_in), b = reinterpret_cast<uintptr_t>(sf_out);
+    if (a != b && a < b + bytes && b < a + bytes)
+        return NVFP4_ERR_INVALID_ARG;        // partial overlap
+    int sms = 0;
+    if ((st = device_setup(&sms)) != NVFP4_OK)
+        return st;
+    convert::HarmonizeParams hp;
+    memset(&hp, 0, sizeof hp);
+    hp.sf_in = sf_in;
+    hp.sf_out = sf_out;
+    hp.rows = n;
+    hp.atoms_k = k / 64;
+    hp.units = static_cast<int64_t>(bytes / 16);
+    hp.nseg = nseg;
+    for (int i = 0; i < nseg; ++i)
+        hp.seg_end[i] = ends[i];
+    hp.gscale = seg_gscales;
+    hp.shared_out = shared_gscale_out;
+    const int64_t blocks = (hp.units + convert::kThreads - 1) / convert::kThreads;
+    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    const int grid = static_cast<int>(blocks < cap ? blocks : cap);
+    return cuda_status(launch(convert::harmonize_kernel, grid, convert::kThreads, 0,
+                              reinterpret_cast<cudaStream_t>(stream), false, hp));
 }
 
 nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream)

@@ -127,6 +127,49 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, 
         : "memory");
 }
 
+// ---------------------------------------------------------------- TMA stores
+
+// Tiled TMA store shared -> global (rows/columns outside the tensor are not written).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int32_t c0, int32_t c1, const void *smem_src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until the bulk stores issued by this thread have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Wait until the bulk stores issued by this thread are complete.
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA, tensor cores).
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Barrier over `nthreads` threads (named barrier `id`) returning whether any
+// participant passed a non-zero flag.
+__device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t nthreads, uint32_t flag)
+{
+    uint32_t any;
+    asm volatile(
+        "{\n\t.reg .pred q, r;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred r, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, r;\n\t}"
+        : "=r"(any)
+        : "r"(flag), "r"(id), "r"(nthreads)
+        : "memory");
+    return any != 0;
+}
+
+__device__ __forceinline__ void bar_sync_named(uint32_t id, uint32_t nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 // Allocate `ncols` tensor-memory columns (power of two >= 32); warp-wide.

@@ -116,6 +116,42 @@ def test_pack_validation(L):
     assert f(FAKE, 0, 128, 128, None, 1, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == nv.ERR_INVALID_ARG
 
 
+def test_dequantize_validation(L):
+    f = L.nvfp4_dequantize
+    assert f(FAKE, FAKE, 4, 96, None, FAKE, 1, FAKE, 96, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, FAKE, -1, 64, None, FAKE, 1, FAKE, 64, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, 64, None, FAKE, 1, FAKE, 32, None) == nv.ERR_INVALID_ARG        # ldy < k
+    assert f(None, FAKE, 4, 64, None, FAKE, 1, FAKE, 64, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, 64, None, None, 1, FAKE, 64, None) == nv.ERR_INVALID_ARG
+    assert f(MIS, FAKE, 4, 64, None, FAKE, 1, FAKE, 64, None) == nv.ERR_MISALIGNED
+    assert f(FAKE, FAKE, 4, 64, None, FAKE, 1, FAKE, 68, None) == nv.ERR_MISALIGNED        # row stride
+    assert f(FAKE, FAKE, 16, 64, _segs(0, 8, 12), FAKE, 2, FAKE, 64, None) == nv.ERR_INVALID_ARG  # last != rows
+    assert f(FAKE, FAKE, 16, 64, _segs(0, 4, 16), FAKE, 2, FAKE, 64, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, FAKE, 0, 64, None, FAKE, 1, FAKE, 64, None) == nv.OK                     # empty: no-op
+
+
+def test_import_scales_validation(L):
+    f = L.nvfp4_import_weight_scales
+    assert f(FAKE, 4, 96, 8, FAKE, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, 4, 128, 4, FAKE, None) == nv.ERR_INVALID_ARG          # ld < k/16
+    assert f(FAKE, 4, 128, 10, FAKE, None) == nv.ERR_MISALIGNED          # ld % 4
+    assert f(FAKE + 2, 4, 128, 8, FAKE + 0x10000, None) == nv.ERR_MISALIGNED
+    assert f(FAKE, 4, 128, 8, FAKE + 8, None) == nv.ERR_MISALIGNED       # output not 16-byte aligned
+    assert f(FAKE, 4, 128, 8, FAKE + 16, None) == nv.ERR_INVALID_ARG     # overlaps the input
+    assert f(None, 4, 128, 8, FAKE, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, 0, 128, 8, FAKE, None) == nv.OK                       # empty: no-op
+
+
+def test_harmonize_validation(L):
+    f = L.nvfp4_harmonize_scales
+    assert f(FAKE, FAKE, 0, 128, None, FAKE, 1, FAKE, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 64, 96, None, FAKE, 1, FAKE, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, FAKE, 64, 128, _segs(0, 16, 60), FAKE, 2, FAKE, None) == nv.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 64, 128, None, FAKE, 1, None, None) == nv.ERR_INVALID_ARG         # no shared-scale slot
+    assert f(MIS, FAKE, 64, 128, None, FAKE, 1, FAKE, None) == nv.ERR_MISALIGNED
+    assert f(FAKE, FAKE + 16, 64, 128, None, FAKE, 1, FAKE, None) == nv.ERR_INVALID_ARG    # partial overlap
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     mod = importlib.import_module("nvfp4_w4a4_block_b200")
