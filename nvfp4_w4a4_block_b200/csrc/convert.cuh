@@ -98,11 +98,14 @@ __device__ __forceinline__ BlockTable block_table(float sd, float s)
         for (int m = 1; m < 8; ++m)
             e[m] = bf16_bits_of_product(e2m1_magnitude(m) * sd, s);   // e2m1 * e4m3 is exact in fp32
     }
+    // e[i] holds a bf16 pattern in its low 16 bits; gather low and high bytes.
+    const uint32_t x01 = __byte_perm(e[0], e[1], 0x5410u), x23 = __byte_perm(e[2], e[3], 0x5410u);
+    const uint32_t x45 = __byte_perm(e[4], e[5], 0x5410u), x67 = __byte_perm(e[6], e[7], 0x5410u);
     BlockTable t;
-    t.lo0 = (e[0] & 0xFFu) | ((e[1] & 0xFFu) << 8) | ((e[2] & 0xFFu) << 16) | ((e[3] & 0xFFu) << 24);
-    t.lo1 = (e[4] & 0xFFu) | ((e[5] & 0xFFu) << 8) | ((e[6] & 0xFFu) << 16) | ((e[7] & 0xFFu) << 24);
-    t.hi0 = (e[0] >> 8) | ((e[1] >> 8) << 8) | ((e[2] >> 8) << 16) | ((e[3] >> 8) << 24);
-    t.hi1 = (e[4] >> 8) | ((e[5] >> 8) << 8) | ((e[6] >> 8) << 16) | ((e[7] >> 8) << 24);
+    t.lo0 = __byte_perm(x01, x23, 0x6420u);
+    t.hi0 = __byte_perm(x01, x23, 0x7531u);
+    t.lo1 = __byte_perm(x45, x67, 0x6420u);
+    t.hi1 = __byte_perm(x45, x67, 0x7531u);
     return t;
 }
 
@@ -132,47 +135,80 @@ struct ExpandParams {
     const float *gscale;       // [nseg] device
 };
 
-// One tile = 128 rows x 64 elements = one 512-byte scale atom.  Thread t owns
-// 32 elements (two blocks) of row t/2: 16 bytes of codes in, 64 bytes out.
+// One tile = 128 rows x 64 elements = one 512-byte scale atom.  Two phases per
+// tile:
+//   1. thread t builds the look-up tables of the two blocks (columns 2(t&1),
+//      2(t&1)+1 of the atom) of row t/2 into shared memory (16 bytes each);
+//   2. thread t expands 8 consecutive elements (4 bytes of codes -> one 16-byte
+//      bf16 store) in each of the rows t/8 + 32j, j = 0..3, so a warp's store
+//      covers four whole 128-byte row segments.
+// The codes and scales of the next tile are loaded before the current tile is
+// expanded.
 __global__ void __launch_bounds__(kThreads) expand_kernel(ExpandParams p)
 {
     __shared__ float s_scale[kMaxSeg];
+    __shared__ uint4 s_tab[128 * 4];              // [row][block]: lo0, lo1, hi0, hi1
     if (threadIdx.x < kMaxSeg)
         s_scale[threadIdx.x] = threadIdx.x < static_cast<unsigned>(p.nseg) ? p.gscale[threadIdx.x] : 0.0f;
     __syncthreads();
-    const int r_in = threadIdx.x >> 1;          // row inside the tile
-    const int half = threadIdx.x & 1;           // which 32 elements of the 64
+    const int g = threadIdx.x & 7;              // phase 2: 8-element group inside the 64 columns
+    const int rsub = threadIdx.x >> 3;          // phase 2: row inside each 32-row quarter
+    const int trow = threadIdx.x >> 1;          // phase 1: row of this thread's two blocks
+    const int tpair = threadIdx.x & 1;          // phase 1: blocks 2*tpair, 2*tpair + 1
     const int64_t tiles = p.row_tiles * p.col_tiles;
     const int64_t kh = p.k >> 1;
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+
+    auto load = [&](int64_t t, uint32_t &sf2, uint32_t (&codes)[4]) {
         const int64_t rt = t / p.col_tiles, ct = t - rt * p.col_tiles;
-        const int64_t row = rt * 128 + r_in;
-        if (row >= p.rows)
-            continue;
-        const uint4 codes = __ldg(reinterpret_cast<const uint4 *>(p.q + row * kh + ct * 32 + half * 16));
-        const uint8_t *atom = p.sf + (rt * p.col_tiles + ct) * 512 + (r_in & 31) * 16 + (r_in >> 5) * 4 + half * 2;
-        const uint32_t sf2 = __ldg(reinterpret_cast<const uint16_t *>(atom));
-        int seg = 0;
+        sf2 = __ldg(reinterpret_cast<const uint16_t *>(p.sf + t * 512 + (trow & 31) * 16 + (trow >> 5) * 4 +
+                                                       tpair * 2));
 #pragma unroll
-        for (int i = 0; i < kMaxSeg - 1; ++i)
-            seg += (i + 1 < p.nseg && row >= p.seg_end[i]) ? 1 : 0;
-        const float s = s_scale[seg];
-        const BlockTable t0 = block_table(e4m3_to_f32(sf2 & 0xFFu), s);
-        const BlockTable t1 = block_table(e4m3_to_f32(sf2 >> 8), s);
-        uint4 o0, o1, o2, o3;
-        expand4(t0, codes.x, o0.x, o0.y);
-        expand4(t0, codes.x >> 16, o0.z, o0.w);
-        expand4(t0, codes.y, o1.x, o1.y);
-        expand4(t0, codes.y >> 16, o1.z, o1.w);
-        expand4(t1, codes.z, o2.x, o2.y);
-        expand4(t1, codes.z >> 16, o2.z, o2.w);
-        expand4(t1, codes.w, o3.x, o3.y);
-        expand4(t1, codes.w >> 16, o3.z, o3.w);
-        uint4 *dst = reinterpret_cast<uint4 *>(p.y + row * p.ldy + ct * 64 + half * 32);
-        dst[0] = o0;
-        dst[1] = o1;
-        dst[2] = o2;
-        dst[3] = o3;
+        for (int j = 0; j < 4; ++j) {
+            const int64_t row = rt * 128 + j * 32 + rsub;
+            codes[j] = row < p.rows ? __ldg(reinterpret_cast<const uint32_t *>(p.q + row * kh + ct * 32 + g * 4)) : 0u;
+        }
+    };
+
+    int64_t t = blockIdx.x;
+    uint32_t sf2 = 0, codes[4] = {0u, 0u, 0u, 0u};
+    if (t < tiles)
+        load(t, sf2, codes);
+    for (; t < tiles; t += gridDim.x) {
+        const int64_t rt = t / p.col_tiles, ct = t - rt * p.col_tiles;
+        // phase 1: tables of this thread's two blocks
+        {
+            const int64_t row = rt * 128 + trow;
+            int seg = 0;
+            if (p.nseg > 1) {
+#pragma unroll
+                for (int i = 0; i < kMaxSeg - 1; ++i)
+                    seg += (i + 1 < p.nseg && row >= p.seg_end[i]) ? 1 : 0;
+            }
+            const float s = s_scale[seg];
+            const BlockTable b0 = block_table(e4m3_to_f32(sf2 & 0xFFu), s);
+            const BlockTable b1 = block_table(e4m3_to_f32(sf2 >> 8), s);
+            s_tab[trow * 4 + tpair * 2] = make_uint4(b0.lo0, b0.lo1, b0.hi0, b0.hi1);
+            s_tab[trow * 4 + tpair * 2 + 1] = make_uint4(b1.lo0, b1.lo1, b1.hi0, b1.hi1);
+        }
+        uint32_t cur[4] = {codes[0], codes[1], codes[2], codes[3]};
+        if (t + gridDim.x < tiles)
+            load(t + gridDim.x, sf2, codes);     // next tile's loads in flight during the expansion
+        __syncthreads();
+        // phase 2: expansion, coalesced stores
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int r = j * 32 + rsub;
+            const int64_t row = rt * 128 + r;
+            if (row < p.rows) {
+                const uint4 tv = s_tab[r * 4 + (g >> 1)];
+                const BlockTable tb = {tv.x, tv.y, tv.z, tv.w};
+                uint4 o;
+                expand4(tb, cur[j], o.x, o.y);
+                expand4(tb, cur[j] >> 16, o.z, o.w);
+                *reinterpret_cast<uint4 *>(p.y + row * p.ldy + ct * 64 + g * 8) = o;
+            }
+        }
+        __syncthreads();                         // s_tab is rewritten by the next tile
     }
 }
 
@@ -186,29 +222,36 @@ struct ImportParams {
     int64_t col_groups;             // ceil(atoms_k / 16)
 };
 
-// One tile = 128 rows x 64 scale columns: rows are read as 4-byte words (one
-// atom's four columns) and the 16 atoms leave as one contiguous 8 KB run.
+
+// One tile = 128 rows x 64 scale columns (16 atoms).  The rows are read as
+// 4-byte words (one atom's four columns), 16 words per row, two rows per warp
+// instruction; they are transposed through shared memory (row stride 17 words:
+// no bank conflicts) and the 16 atoms leave as one contiguous 8 KB run of
+// 16-byte stores.
 __global__ void __launch_bounds__(kThreads) import_scales_kernel(ImportParams p)
 {
+    __shared__ uint32_t tile[128][17];
     const int64_t tiles = p.row_tiles * p.col_groups;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int64_t rt = t / p.col_groups, cg = t - rt * p.col_groups;
         const int64_t a0 = cg * 16;
         const int natoms = static_cast<int>(p.atoms_k - a0 < 16 ? p.atoms_k - a0 : 16);
-        // 16 atoms x 32 words of 16 bytes; thread handles word w of atom a.
-        for (int i = threadIdx.x; i < natoms * 32; i += blockDim.x) {
-            const int a = i >> 5, w = i & 31;     // atom, and row-in-quarter (r % 32)
-            uint32_t v[4];
+        const int w = threadIdx.x & 15;
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-                const int64_t row = rt * 128 + qd * 32 + w;
-                v[qd] = row < p.rows
-                            ? __ldg(reinterpret_cast<const uint32_t *>(p.lin + row * p.ld + (a0 + a) * 4))
-                            : 0u;
-            }
-            *reinterpret_cast<uint4 *>(p.sf + (rt * p.atoms_k + a0 + a) * 512 + w * 16) =
-                make_uint4(v[0], v[1], v[2], v[3]);
+        for (int r0 = 0; r0 < 128; r0 += kThreads / 16) {
+            const int r = r0 + (threadIdx.x >> 4);
+            const int64_t row = rt * 128 + r;
+            tile[r][w] = (row < p.rows && w < natoms)
+                             ? __ldg(reinterpret_cast<const uint32_t *>(p.lin + row * p.ld + (a0 + w) * 4))
+                             : 0u;
         }
+        __syncthreads();
+        for (int i = threadIdx.x; i < natoms * 32; i += blockDim.x) {
+            const int a = i >> 5, r = i & 31;        // atom, and row inside a 32-row quarter
+            *reinterpret_cast<uint4 *>(p.sf + (rt * p.atoms_k + a0 + a) * 512 + r * 16) =
+                make_uint4(tile[r][a], tile[32 + r][a], tile[64 + r][a], tile[96 + r][a]);
+        }
+        __syncthreads();
     }
 }
 

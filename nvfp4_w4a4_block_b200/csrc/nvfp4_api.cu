@@ -44,11 +44,13 @@ struct DeviceInfo {
     nvfp4_status status = NVFP4_OK;
     int sms = 0;
     int tile_quant_ctas_per_sm = 1;
+    int expand_ctas_per_sm = 1;
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[64];
 thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
+thread_local int g_expand_ctas = 148;       // resident expansion CTAs on the current device
 constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder below, tiled encoder above
 constexpr int64_t kSelfAmaxElems = int64_t(1) << 14;     // dynamic scale reduced inside the encoder below
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -125,12 +127,18 @@ nvfp4_status device_setup(int *sms)
             cudaSuccess)
             return NVFP4_ERR_CUDA;
         d.tile_quant_ctas_per_sm = occ > 0 ? occ : 1;
+        occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, convert::expand_kernel, convert::kThreads, 0) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        d.expand_ctas_per_sm = occ > 0 ? occ : 1;
         d.sms = sm;
         d.status = NVFP4_OK;
         d.ready = true;
     }
     *sms = d.sms;
     g_tile_quant_ctas = d.sms * d.tile_quant_ctas_per_sm;
+    g_expand_ctas = d.sms * d.expand_ctas_per_sm;
     return d.status;
 }
 
@@ -708,8 +716,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, int64_t rows,
         ep.seg_end[i] = ends[i];
     ep.gscale = seg_gscales;
     const int64_t tiles = ep.row_tiles * ep.col_tiles;
-    const int64_t cap = static_cast<int64_t>(sms) * 8;
-    const int grid = static_cast<int>(tiles < cap ? tiles : cap);
+    const int grid = static_cast<int>(tiles < g_expand_ctas ? tiles : g_expand_ctas);
     return cuda_status(launch(convert::expand_kernel, grid, convert::kThreads, 0,
                               reinterpret_cast<cudaStream_t>(stream), false, ep));
 }
