@@ -231,6 +231,25 @@ def committed_traffic(kernel: str, workload: str):
         return None
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, device="cpu") -> float:
+    """The largest value of x over all ranks of the default process group (x
+    itself without one).  Every rank must call it, in the same order."""
+    import torch
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, step_bytes: int, steps: int, ms_max: float) -> float:
+    """Aggregate throughput of `world` replicas that each moved step_bytes per
+    step for `steps` steps, over the slowest rank's time."""
+    return world * step_bytes * steps / (ms_max * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------------------- workload bytes
 
 def decode_call_bytes(m, n, k, dynamic=True, gemm_only=False):
@@ -335,12 +354,9 @@ def run_nvfp4(args, rank, world, local_rank):
     ms_total = e0.elapsed_time(e1)
     if nv.get_device_error() != nv.OK:
         raise RuntimeError("device error in the timed region")
-    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms_total, "cuda")
     ms_per_step = ms_max / args.steps
-    value = world * step_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, args.steps, ms_max)
     del graphs
 
     # ---- dominant kernel: the GEMM alone, per M.  A graph holds `copies` launches
