@@ -208,25 +208,30 @@ def time_graph(g, reps, per_replay):
     return e0.elapsed_time(e1) / (reps * per_replay)
 
 
-def kernel_source_hash():
+def kernel_source_hash(files):
+    """Hash of a kernel's own source files (under the package's csrc/)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nvfp4_w4a4_block_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    for name in files:
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
 
 
-def committed_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+DECODE_KERNEL_FILES = ("gemm_decode.cuh", "sm100_ptx.cuh")
+
+
+def committed_traffic(summary: str, files):
+    """DRAM bytes per launch recorded in a committed ncu summary under profiles/
+    (its 'dram bytes per launch' and 'kernel source hash' lines), if that capture
+    was taken on the kernel's current sources; else None."""
+    import re
     try:
-        d = json.load(open(path))
-        e = d[kernel][workload]
-        if e.get("source_hash") != kernel_source_hash():
+        text = open(os.path.join(ROOT, "profiles", summary)).read()
+        b = re.search(r"dram bytes per launch:\s*([0-9]+)", text)
+        hsh = re.search(r"kernel source hash:\s*([0-9a-f]+)", text)
+        if not b or not hsh or hsh.group(1) != kernel_source_hash(files):
             return None
-        return float(e["dram_bytes_per_launch"])
+        return int(b.group(1))
     except Exception:
         return None
 
@@ -393,10 +398,10 @@ def run_nvfp4(args, rank, world, local_rank):
                              call_static_scale_us=round(ts * 1e3, 3),
                              gemm_bytes=gb, call_bytes=fb)
     gm = per_m[str(mmax)]
-    roofline = dict(bound="hbm", kernel="nvfp4_gemm_kernel", workload=f"decode M={mmax}",
+    roofline = dict(bound="hbm", kernel="nvfp4_gemm_decode_kernel", workload=f"decode M={mmax}",
                     achieved=round(gm["gemm_gbs"], 1), peak=peaks["hbm_gbs"], unit="GB/s",
                     frac=round(gm["gemm_gbs"] / peaks["hbm_gbs"], 4),
-                    traffic=committed_traffic("nvfp4_gemm_kernel", f"decode_M{mmax}"),
+                    traffic=committed_traffic(f"nvfp4_gemm_decode_kernel_m{mmax}.md", DECODE_KERNEL_FILES),
                     algorithmic_bytes_per_launch=gm["gemm_bytes"], peak_source=peaks["source"])
 
     # ---- end to end through host buffers (pinned), H2D of X and D2H of Y inside the region

@@ -135,33 +135,31 @@ struct ExpandParams {
     const float *gscale;       // [nseg] device
 };
 
-// One tile = 128 rows x 64 elements = one 512-byte scale atom.  Two phases per
-// tile:
-//   1. thread t builds the look-up tables of the two blocks (columns 2(t&1),
-//      2(t&1)+1 of the atom) of row t/2 into shared memory (16 bytes each);
-//   2. thread t expands 8 consecutive elements (4 bytes of codes -> one 16-byte
-//      bf16 store) in each of the rows t/8 + 32j, j = 0..3, so a warp's store
-//      covers four whole 128-byte row segments.
-// The codes and scales of the next tile are loaded before the current tile is
-// expanded.
+// A block's eight bf16 magnitudes depend only on its scale byte and its
+// segment's global scale, so each CTA first tabulates them for all 128
+// non-negative E4M3 codes of every segment (16 bytes per entry, at most 16 KB of
+// shared memory).  One tile = 128 rows x 64 elements = one 512-byte scale atom;
+// thread t expands 8 consecutive elements (4 bytes of codes -> one 16-byte bf16
+// store) in each of the rows t/8 + 32j, j = 0..3, so a warp's store covers four
+// whole 128-byte row segments; its four scale bytes sit in one 16-byte word of
+// the atom.  The next tile's codes and scales are loaded before the current
+// tile is expanded.  A scale byte with its sign bit set negates the block.
 __global__ void __launch_bounds__(kThreads) expand_kernel(ExpandParams p)
 {
-    __shared__ float s_scale[kMaxSeg];
-    __shared__ uint4 s_tab[128 * 4];              // [row][block]: lo0, lo1, hi0, hi1
-    if (threadIdx.x < kMaxSeg)
-        s_scale[threadIdx.x] = threadIdx.x < static_cast<unsigned>(p.nseg) ? p.gscale[threadIdx.x] : 0.0f;
+    __shared__ uint4 s_lut[kMaxSeg * 128];
+    for (int idx = threadIdx.x; idx < p.nseg * 128; idx += blockDim.x) {
+        const BlockTable tb = block_table(e4m3_to_f32(static_cast<uint32_t>(idx & 127)), p.gscale[idx >> 7]);
+        s_lut[idx] = make_uint4(tb.lo0, tb.lo1, tb.hi0, tb.hi1);
+    }
     __syncthreads();
-    const int g = threadIdx.x & 7;              // phase 2: 8-element group inside the 64 columns
-    const int rsub = threadIdx.x >> 3;          // phase 2: row inside each 32-row quarter
-    const int trow = threadIdx.x >> 1;          // phase 1: row of this thread's two blocks
-    const int tpair = threadIdx.x & 1;          // phase 1: blocks 2*tpair, 2*tpair + 1
+    const int g = threadIdx.x & 7;              // 8-element group inside the 64 columns
+    const int rsub = threadIdx.x >> 3;          // row inside each 32-row quarter
     const int64_t tiles = p.row_tiles * p.col_tiles;
     const int64_t kh = p.k >> 1;
-
-    auto load = [&](int64_t t, uint32_t &sf2, uint32_t (&codes)[4]) {
-        const int64_t rt = t / p.col_tiles, ct = t - rt * p.col_tiles;
-        sf2 = __ldg(reinterpret_cast<const uint16_t *>(p.sf + t * 512 + (trow & 31) * 16 + (trow >> 5) * 4 +
-                                                       tpair * 2));
+    // (row tile, column tile) advance by a precomputed step: no division in the loop.
+    const int64_t step_r = gridDim.x / p.col_tiles, step_c = gridDim.x % p.col_tiles;
+    auto load = [&](int64_t t, int64_t rt, int64_t ct, uint4 &sfw, uint32_t (&codes)[4]) {
+        sfw = __ldg(reinterpret_cast<const uint4 *>(p.sf + t * 512 + rsub * 16));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int64_t row = rt * 128 + j * 32 + rsub;
@@ -170,45 +168,47 @@ __global__ void __launch_bounds__(kThreads) expand_kernel(ExpandParams p)
     };
 
     int64_t t = blockIdx.x;
-    uint32_t sf2 = 0, codes[4] = {0u, 0u, 0u, 0u};
+    int64_t rt = t / p.col_tiles, ct = t % p.col_tiles;
+    uint4 sfw = make_uint4(0, 0, 0, 0);
+    uint32_t codes[4] = {0u, 0u, 0u, 0u};
     if (t < tiles)
-        load(t, sf2, codes);
+        load(t, rt, ct, sfw, codes);
     for (; t < tiles; t += gridDim.x) {
-        const int64_t rt = t / p.col_tiles, ct = t - rt * p.col_tiles;
-        // phase 1: tables of this thread's two blocks
-        {
-            const int64_t row = rt * 128 + trow;
+        int64_t nrt = rt + step_r, nct = ct + step_c;
+        if (nct >= p.col_tiles) {
+            nct -= p.col_tiles;
+            ++nrt;
+        }
+        const uint32_t sfv[4] = {sfw.x, sfw.y, sfw.z, sfw.w};
+        const uint32_t cur[4] = {codes[0], codes[1], codes[2], codes[3]};
+        if (t + gridDim.x < tiles)
+            load(t + gridDim.x, nrt, nct, sfw, codes);   // next tile's loads in flight during the expansion
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t row = rt * 128 + j * 32 + rsub;
+            if (row >= p.rows)
+                continue;
             int seg = 0;
             if (p.nseg > 1) {
 #pragma unroll
                 for (int i = 0; i < kMaxSeg - 1; ++i)
                     seg += (i + 1 < p.nseg && row >= p.seg_end[i]) ? 1 : 0;
             }
-            const float s = s_scale[seg];
-            const BlockTable b0 = block_table(e4m3_to_f32(sf2 & 0xFFu), s);
-            const BlockTable b1 = block_table(e4m3_to_f32(sf2 >> 8), s);
-            s_tab[trow * 4 + tpair * 2] = make_uint4(b0.lo0, b0.lo1, b0.hi0, b0.hi1);
-            s_tab[trow * 4 + tpair * 2 + 1] = make_uint4(b1.lo0, b1.lo1, b1.hi0, b1.hi1);
+            const uint32_t sb = (sfv[j] >> (8 * (g >> 1))) & 0xFFu;
+            const uint4 tv = s_lut[seg * 128 + (sb & 0x7Fu)];
+            const BlockTable tb = {tv.x, tv.y, tv.z, tv.w};
+            const uint32_t neg = (sb & 0x80u) ? 0x80008000u : 0u;
+            uint4 o;
+            expand4(tb, cur[j], o.x, o.y);
+            expand4(tb, cur[j] >> 16, o.z, o.w);
+            o.x ^= neg;
+            o.y ^= neg;
+            o.z ^= neg;
+            o.w ^= neg;
+            *reinterpret_cast<uint4 *>(p.y + row * p.ldy + ct * 64 + g * 8) = o;
         }
-        uint32_t cur[4] = {codes[0], codes[1], codes[2], codes[3]};
-        if (t + gridDim.x < tiles)
-            load(t + gridDim.x, sf2, codes);     // next tile's loads in flight during the expansion
-        __syncthreads();
-        // phase 2: expansion, coalesced stores
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int r = j * 32 + rsub;
-            const int64_t row = rt * 128 + r;
-            if (row < p.rows) {
-                const uint4 tv = s_tab[r * 4 + (g >> 1)];
-                const BlockTable tb = {tv.x, tv.y, tv.z, tv.w};
-                uint4 o;
-                expand4(tb, cur[j], o.x, o.y);
-                expand4(tb, cur[j] >> 16, o.z, o.w);
-                *reinterpret_cast<uint4 *>(p.y + row * p.ldy + ct * 64 + g * 8) = o;
-            }
-        }
-        __syncthreads();                         // s_tab is rewritten by the next tile
+        rt = nrt;
+        ct = nct;
     }
 }
 
@@ -232,8 +232,9 @@ __global__ void __launch_bounds__(kThreads) import_scales_kernel(ImportParams p)
 {
     __shared__ uint32_t tile[128][17];
     const int64_t tiles = p.row_tiles * p.col_groups;
+    const int64_t step_r = gridDim.x / p.col_groups, step_c = gridDim.x % p.col_groups;
+    int64_t rt = blockIdx.x / p.col_groups, cg = blockIdx.x % p.col_groups;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const int64_t rt = t / p.col_groups, cg = t - rt * p.col_groups;
         const int64_t a0 = cg * 16;
         const int natoms = static_cast<int>(p.atoms_k - a0 < 16 ? p.atoms_k - a0 : 16);
         const int w = threadIdx.x & 15;
@@ -252,6 +253,12 @@ __global__ void __launch_bounds__(kThreads) import_scales_kernel(ImportParams p)
                 make_uint4(tile[r][a], tile[32 + r][a], tile[64 + r][a], tile[96 + r][a]);
         }
         __syncthreads();
+        rt += step_r;
+        cg += step_c;
+        if (cg >= p.col_groups) {
+            cg -= p.col_groups;
+            ++rt;
+        }
     }
 }
 

@@ -161,6 +161,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         uint32_t phase = 0;
         bool ok = true;
         const uint32_t bar0 = map_to_rank(smem_u32(&full[0]), 0);
+        const uint64_t keep = policy_evict_last();       // operand tiles are re-read by other pairs
         for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
             const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
             const int row_a = mb * BM + static_cast<int>(rank) * 128;
@@ -173,8 +174,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (elect_one()) {
                     if (rank == 0)
                         mbar_arrive_expect_tx(&full[stage], TX_BYTES);
-                    tma_load_2d_pair(smem + OFF_A + stage * A_BYTES, &tm_a, ks * (BK / 2), row_a, bar);
-                    tma_load_2d_pair(smem + OFF_B + stage * B_BYTES, &tm_b, ks * (BK / 2), row_b, bar);
+                    tma_load_2d_pair_hint(smem + OFF_A + stage * A_BYTES, &tm_a, ks * (BK / 2), row_a, bar, keep);
+                    tma_load_2d_pair_hint(smem + OFF_B + stage * B_BYTES, &tm_b, ks * (BK / 2), row_b, bar, keep);
                     tma_load_3d_pair(smem + OFF_SFA + stage * SFA_BYTES, &tm_sfa, 0, ks * KB,
                                      mb * 2 + static_cast<int>(rank), bar);
                     tma_load_3d_pair(smem + OFF_SFB + stage * SFB_BYTES, &tm_sfb, 0, ks * KB, nb * 2, bar);
@@ -279,6 +280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const bool f32_out = (p.flags & FLAG_F32_OUT) != 0;
         const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
         uint8_t *stg = smem + OFF_STG;
+        const uint64_t stream_out = policy_evict_first();  // output tiles are written once
         uint32_t acc_phase = 0;
         for (int tile = pair_id; tile < num_tiles; tile += npairs) {
             const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
@@ -342,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         for (int sub = 0; sub < 2; ++sub) {
                             const int col = n0 + round * 128 + sub * 64;
                             if (col < p.n)
-                                tma_store_2d(&tm_y, col, m0, stg + sub * STG_SUB);
+                                tma_store_2d_hint(&tm_y, col, m0, stg + sub * STG_SUB, stream_out);
                         }
                         bulk_commit_group();
                     }

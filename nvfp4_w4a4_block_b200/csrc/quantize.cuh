@@ -377,7 +377,7 @@ __device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b)
 }
 
 // One 16-element block (8 words of bf16 pairs) -> 8 bytes of codes, scale byte.
-__device__ __forceinline__ uint2 encode_block16(const uint32_t (&w)[8], float s, float dg, uint32_t &sb_out)
+__device__ __forceinline__ uint2 encode_block16(const uint32_t (&w)[8], const float *rcp, float dg, uint32_t &sb_out)
 {
     const uint32_t msk = 0x7FFF7FFFu;
     uint32_t a = __vmaxu2(__vmaxu2(w[0] & msk, w[1] & msk), __vmaxu2(w[2] & msk, w[3] & msk));
@@ -386,8 +386,7 @@ __device__ __forceinline__ uint2 encode_block16(const uint32_t (&w)[8], float s,
     const float bmax = __uint_as_float(max(c >> 16, c & 0xFFFFu) << 16);
     const float sbf = (dg == 0.0f) ? 0.0f : fminf(__fdiv_rn(bmax, dg), 448.0f);
     const uint32_t sb = f32_to_e4m3(sbf);
-    const float d = __fmul_rn(e4m3_to_f32(sb), s);
-    const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX);
+    const float r = rcp[sb];                 // min(1 / (value(sb) * s), FLT_MAX), or 0
     const uint64_t rr = (static_cast<uint64_t>(__float_as_uint(r)) << 32) | __float_as_uint(r);
     float v[16];
 #pragma unroll
@@ -407,6 +406,10 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(TileQuantP
     __shared__ float s_scale[kMaxSeg];
     __shared__ float s_dg[kMaxSeg];
     __shared__ __align__(16) uint32_t s_atom[2][128];
+    // Per segment, the element multiplier of every block-scale code c:
+    // r = min(1 / (value(c) * s), FLT_MAX), 0 when value(c) * s == 0 -- the same
+    // fp32 operations as computing it per block, done once per CTA.
+    __shared__ float s_rcp[kMaxSeg][128];
     const int lane = threadIdx.x & 31;
 
     pdl_wait_prerequisites();
@@ -439,6 +442,11 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(TileQuantP
             if (blockIdx.x == 0)
                 p.scale_out[seg] = s;
         }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < p.nseg * 128; idx += blockDim.x) {
+        const float d = __fmul_rn(e4m3_to_f32(static_cast<uint32_t>(idx & 127)), s_scale[idx >> 7]);
+        s_rcp[idx >> 7][idx & 127] = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX);
     }
     __syncthreads();
 
@@ -481,16 +489,19 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(TileQuantP
         const int64_t row = rt * 128 + rl;
         const bool valid = row < p.rows;
         int seg = 0;
+        if (p.nseg > 1) {
 #pragma unroll
-        for (int s = 0; s < kMaxSeg - 1; ++s)
-            seg += (s + 1 < p.nseg && row >= p.seg_end[s]) ? 1 : 0;
-        const float s = s_scale[seg], dg = s_dg[seg];
+            for (int s = 0; s < kMaxSeg - 1; ++s)
+                seg += (s + 1 < p.nseg && row >= p.seg_end[s]) ? 1 : 0;
+        }
+        const float *rcp = s_rcp[seg];
+        const float dg = s_dg[seg];
 
         const uint32_t w0[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
         const uint32_t w1[8] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
         uint32_t sb0, sb1;
-        const uint2 c0 = encode_block16(w0, s, dg, sb0);
-        const uint2 c1 = encode_block16(w1, s, dg, sb1);
+        const uint2 c0 = encode_block16(w0, rcp, dg, sb0);
+        const uint2 c1 = encode_block16(w1, rcp, dg, sb1);
         if (valid)
             *reinterpret_cast<uint4 *>(p.q + row * (p.k >> 1) + ct * 32 + half * 16) = make_uint4(c0.x, c0.y, c1.x, c1.y);
 

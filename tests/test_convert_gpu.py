@@ -73,7 +73,20 @@ def test_dequantize_random_codes_and_scales_bit_exact(nv, rows, k, nseg):
     assert np.array_equal(_bits(y), ref)
 
 
-@pytest.mark.parametrize("s", [2.0 ** -126, 1e-40, 3.0e-39, 2.0 ** 100, 7.7e33, 1.0 / 3.0])
+def test_dequantize_negative_scale_bytes_bit_exact(nv):
+    """E4M3 block-scale bytes with the sign bit set (never written by the
+    quantizer, possible in an imported checkpoint) negate their block."""
+    import torch
+    rng = np.random.default_rng(13)
+    rows, k = 136, 256
+    q = rng.integers(0, 256, (rows, k // 2), dtype=np.uint8)
+    sf = rng.integers(0, 0x7F, (rows, k // 16), dtype=np.uint8) | (rng.integers(0, 2, (rows, k // 16)) * 0x80).astype(np.uint8)
+    y = nv.dequantize(_u8(q), _u8(oracle.sf_to_physical(sf, k)), k, _f32([0.37]))
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y), oracle.dequantize_bf16(q, sf, np.float32(0.37)))
+
+
+@pytest.mark.parametrize("s", [2.0 ** -126, 1e-40, 3.0e-39, 2.0 ** 100, 7.7e33, 2e35, 1.0 / 3.0])
 def test_dequantize_extreme_global_scales_bit_exact(nv, s):
     """Products in bf16's subnormal range, at the fp32 underflow edge and near
     overflow all take the one correct rounding."""
