@@ -410,14 +410,39 @@ def run_nvfp4(args, rank, world, local_rank):
     dx = {m: torch.empty_like(xs[m]) for m in ms}
 
     ctr = [0]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_step():
-        for m in ms:
+        # The step's three calls pipelined over three streams: all inputs go up on
+        # s_in, the layer runs on the current stream as each input lands, and each
+        # result comes back on s_out while the next call computes.  The step ends
+        # when the current stream has waited for the last read-back, and the next
+        # step's copies start only after that (its buffers are then free).
+        cur = torch.cuda.current_stream()
+        start = torch.cuda.Event()
+        start.record(cur)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        landed = []
+        with torch.cuda.stream(s_in):
+            for m in ms:
+                dx[m].copy_(hx[m], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(s_in)
+                landed.append(ev)
+        for j, m in enumerate(ms):
             pw = pws[ctr[0] % copies]
             ctr[0] += 1
-            dx[m].copy_(hx[m], non_blocking=True)
+            cur.wait_event(landed[j])
             nv.linear_fused(dx[m], pw, out=ys[m], ws=wss[m])
-            hy[m].copy_(ys[m], non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(cur)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                hy[m].copy_(ys[m], non_blocking=True)
+        back = torch.cuda.Event()
+        back.record(s_out)
+        cur.wait_event(back)
 
     te = time_reps(e2e_step, max(10, min(args.steps, 200)), 3)
     e2e_ms = statistics.median(te)

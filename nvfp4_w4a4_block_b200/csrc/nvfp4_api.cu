@@ -52,7 +52,9 @@ DeviceInfo g_dev[64];
 thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
 thread_local int g_expand_ctas = 148;       // resident expansion CTAs on the current device
 constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder below, tiled encoder above
-constexpr int64_t kSelfAmaxElems = int64_t(1) << 14;     // dynamic scale reduced inside the encoder below
+// Dynamic scale for decode-sized activations: one cluster launch holds the whole
+// tensor in registers (quantize_cluster_kernel) up to this many elements.
+constexpr int64_t kClusterQuantElems = int64_t(kClusterCtas) * kClusterThreads * kClusterUnits * 8;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -202,20 +204,18 @@ int quant_grid(int sms, int64_t rows, int64_t k)
     return static_cast<int>(g < 1 ? 1 : g);
 }
 
-// Quantization of [rows, k] (rows split into segments).  Small tensors (at most
-// 2^20 elements, one segment) use one kernel that also reduces the dynamic amax;
-// larger ones run the amax pass (dynamic mode) and the tiled encoder.
+// Quantization of [rows, k] (rows split into segments).  One segment, dynamic
+// scale, at most 65536 elements (decode): one cluster launch reduces the amax
+// and encodes.  Up to 2^20 elements: the per-unit encoder, after an amax pass in
+// dynamic mode.  Larger (or several segments): amax passes and the tiled encoder.
 nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx, const int64_t *seg_ends, int nseg,
                              const float *static_scale, float *scale_out, uint8_t *q, uint8_t *sf,
                              uint32_t *partials, int sms, cudaStream_t stream)
 {
     const int ga = amax_grid(sms, rows, k);
     if (nseg == 1 && rows * k <= kSmallQuantElems) {
-        // Tiny tensors (decode): in dynamic mode every CTA of the single encoder
-        // launch reduces the whole tensor itself (few CTAs, so few redundant reads);
-        // up to 2^20 elements an amax pass precedes the per-unit encoder.
-        const bool self_amax = static_scale == nullptr && rows * k <= kSelfAmaxElems;
-        if (static_scale == nullptr && !self_amax) {
+        const bool cluster = static_scale == nullptr && rows * k <= kClusterQuantElems;
+        if (static_scale == nullptr && !cluster) {
             AmaxParams ap;
             ap.x = static_cast<const uint16_t *>(x);
             ap.row_begin = 0;
@@ -242,10 +242,9 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
         qp.partial = partials;
         qp.npartial = ga;
         qp.scale_out = scale_out;
-        qp.self_amax = self_amax ? 1 : 0;
-        int grid = quant_grid(sms, rows, k);
-        if (self_amax && grid > 16)
-            grid = 16;
+        if (cluster)
+            return cuda_status(launch(quantize_cluster_kernel, kClusterCtas, kClusterThreads, 0, stream, true, qp));
+        const int grid = quant_grid(sms, rows, k);
         return cuda_status(launch(quantize_kernel, grid, kQuantThreads, 0, stream, true, qp));
     }
     if (static_scale == nullptr) {

@@ -168,7 +168,6 @@ struct QuantParams {
     const uint32_t *partial;     // [nseg][npartial] amax partials (dynamic)
     int npartial;
     float *scale_out;            // [nseg]
-    int self_amax;               // dynamic, one segment: each CTA reduces the whole tensor itself
 };
 
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
@@ -183,47 +182,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
     pdl_wait_prerequisites();
     pdl_launch_dependents();
 
-    // Small tensors in dynamic mode: every CTA reduces the whole (L2-resident)
-    // tensor itself, which saves the separate amax launch and its dependency.
-    __shared__ uint32_t s_red[kQuantThreads / 32];
-    if (p.self_amax) {
-        const int64_t upr0 = p.k >> 3;
-        const int64_t total0 = p.rows * upr0;
-        uint32_t b = 0;
-        // Four independent 16-byte loads in flight per thread per round.
-        for (int64_t u0 = threadIdx.x; u0 < total0; u0 += 4 * blockDim.x) {
-            uint4 v[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int64_t u = u0 + j * blockDim.x;
-                v[j] = u < total0 ? __ldg(reinterpret_cast<const uint4 *>(p.x + (u / upr0) * p.ldx + (u % upr0) * 8))
-                                  : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                b = max(b, absmax_bits8(v[j]));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
-        if (lane == 0)
-            s_red[threadIdx.x >> 5] = b;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t m = 0;
-            for (int w = 0; w < kQuantThreads / 32; ++w)
-                m = max(m, s_red[w]);
-            float s = __fdiv_rn(__uint_as_float(m << 16), 2688.0f);
-            if (m >= 0x7F80u) {
-                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
-                s = 0.0f;
-            }
-            s_scale[0] = s;
-            s_dg[0] = __fmul_rn(s, 6.0f);
-            if (blockIdx.x == 0)
-                p.scale_out[0] = s;
-        }
-    } else if (threadIdx.x < 32 * p.nseg && (threadIdx.x >> 5) < kMaxSeg) {
+    if (threadIdx.x < 32 * p.nseg && (threadIdx.x >> 5) < kMaxSeg) {
         // Per-segment global scale: given, or amax / 2688 from the amax partials.
         const int seg = threadIdx.x >> 5;
         float s;
@@ -335,6 +294,134 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
             wcol -= upr;
             ++wrow;
         }
+    }
+
+    // Zero the scale bytes of the pad rows [rows, rows_pad): 4 bytes per (row, atom).
+    const int64_t pad_words = (p.rows_pad - p.rows) * (p.kb_pad >> 2);
+    for (int64_t i = gtid; i < pad_words; i += nthreads) {
+        const int64_t row = p.rows + i / (p.kb_pad >> 2);
+        const int64_t kb = (i % (p.kb_pad >> 2)) << 2;
+        *reinterpret_cast<uint32_t *>(p.sf + sf_atom_offset(row, kb, p.kb_pad)) = 0u;
+    }
+}
+
+// ------------------------------------------------------------------ encode, one cluster
+
+// Decode-sized activations in dynamic mode, in one launch: a cluster of
+// kClusterCtas CTAs holds the whole tensor in registers (at most
+// kClusterUnits 16-byte units per thread), reduces the absolute maximum over
+// the cluster through distributed shared memory, and encodes from the same
+// registers -- one read of X, no amax pass, no workspace.  Unit-to-lane mapping,
+// arithmetic and stores are those of quantize_kernel.
+constexpr int kClusterCtas = 8;
+constexpr int kClusterThreads = 512;
+constexpr int kClusterUnits = 2;
+
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t cta_rank_in_cluster()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_barrier()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
+    quantize_cluster_kernel(QuantParams p)
+{
+    __shared__ uint32_t s_red[kClusterThreads / 32];
+    __shared__ uint32_t s_cta_max;
+    __shared__ float s_sc[2];
+    const int lane = threadIdx.x & 31;
+
+    pdl_wait_prerequisites();
+    pdl_launch_dependents();
+
+    const int64_t upr = p.k >> 3;
+    const int64_t total = p.rows * upr;
+    const int64_t nthreads = static_cast<int64_t>(kClusterCtas) * kClusterThreads;
+    const int64_t gtid = static_cast<int64_t>(cta_rank_in_cluster()) * kClusterThreads + threadIdx.x;
+    uint4 v[kClusterUnits];
+    uint32_t b = 0;
+#pragma unroll
+    for (int j = 0; j < kClusterUnits; ++j) {
+        const int64_t u = gtid + j * nthreads;
+        v[j] = u < total ? __ldg(reinterpret_cast<const uint4 *>(p.x + (u / upr) * p.ldx + (u % upr) * 8))
+                         : make_uint4(0, 0, 0, 0);
+        b = max(b, absmax_bits8(v[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+    if (lane == 0)
+        s_red[threadIdx.x >> 5] = b;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t m = 0;
+        for (int w = 0; w < kClusterThreads / 32; ++w)
+            m = max(m, s_red[w]);
+        s_cta_max = m;
+    }
+    cluster_barrier();                                   // every CTA's maximum is in its shared memory
+    if (threadIdx.x == 0) {
+        uint32_t m = 0;
+        for (int r = 0; r < kClusterCtas; ++r)
+            m = max(m, ld_shared_cluster_u32(map_to_rank(smem_u32(&s_cta_max), static_cast<uint32_t>(r))));
+        float sv = __fdiv_rn(__uint_as_float(m << 16), 2688.0f);
+        if (m >= 0x7F80u) {
+            if (cta_rank_in_cluster() == 0)
+                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
+            sv = 0.0f;
+        }
+        s_sc[0] = sv;
+        s_sc[1] = __fmul_rn(sv, 6.0f);
+        if (cta_rank_in_cluster() == 0)
+            p.scale_out[0] = sv;
+    }
+    // The peers' maxima have been read: no CTA of the cluster touches another's
+    // shared memory after this barrier, so each may run to its end.
+    cluster_barrier();
+    const float s = s_sc[0], dg = s_sc[1];
+
+#pragma unroll
+    for (int j = 0; j < kClusterUnits; ++j) {
+        const int64_t u = gtid + j * nthreads;
+        if (__shfl_sync(0xFFFFFFFFu, u, 0) >= total)       // warp-uniform: lane 0 holds the warp's first unit
+            break;
+        const bool active = u < total;
+        const int64_t r_ = active ? u / upr : 0;
+        const int64_t c8 = active ? u % upr : 0;
+        uint32_t bm = absmax_bits8(v[j]);
+        bm = max(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
+        const float bmax = __uint_as_float(bm << 16);
+        const float sbf = (dg == 0.0f) ? 0.0f : fminf(__fdiv_rn(bmax, dg), 448.0f);
+        const uint32_t sb = f32_to_e4m3(sbf);
+        const float d = __fmul_rn(e4m3_to_f32(sb), s);
+        const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX);
+        const uint32_t w0 = v[j].x, w1 = v[j].y, w2 = v[j].z, w3 = v[j].w;
+        const uint32_t codes = f32x8_to_e2m1x8(
+            __fmul_rn(bf16lo(w0), r), __fmul_rn(bf16hi(w0), r), __fmul_rn(bf16lo(w1), r),
+            __fmul_rn(bf16hi(w1), r), __fmul_rn(bf16lo(w2), r), __fmul_rn(bf16hi(w2), r),
+            __fmul_rn(bf16lo(w3), r), __fmul_rn(bf16hi(w3), r));
+        if (active)
+            p.q[r_ * upr + c8] = codes;
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sb, 6);
+        if (active && (lane & 7) == 0)
+            *reinterpret_cast<uint32_t *>(p.sf + sf_atom_offset(r_, c8 >> 1, p.kb_pad)) =
+                sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
     }
 
     // Zero the scale bytes of the pad rows [rows, rows_pad): 4 bytes per (row, atom).

@@ -155,6 +155,29 @@ def test_quantize_nonfinite_sets_device_error(nv):
     assert nv.get_device_error() == nv.OK
 
 
+@pytest.mark.parametrize("m,k", [(4, 5120), (8, 5120), (12, 5120), (13, 5120), (64, 5120), (3, 17408),
+                                 (4, 17408), (1, 65536), (1, 65600)])
+def test_quantize_decode_sizes_around_the_one_launch_limit(nv, m, k):
+    """Dynamic-scale activations up to 65536 elements are quantized in one
+    cluster launch (the whole tensor held in registers); just above that the
+    amax pass and the per-unit encoder take over.  Both sides of the limit."""
+    x, _, _ = W.random_case(33, m, 8, k)
+    _compare(nv, x)
+
+
+@pytest.mark.parametrize("m,k", [(8, 5120), (12, 5120)])
+def test_quantize_nonfinite_in_the_one_launch_path(nv, m, k):
+    import torch
+    x, _, _ = W.random_case(34, m, 8, k)
+    x = x.copy()
+    x[m - 1, k - 3] = 0xFF80                             # -inf in the last unit
+    nv.quantize_act(to_cuda_bf16(x))
+    assert nv.get_device_error() == nv.ERR_NONFINITE
+    nv.quantize_act(to_cuda_bf16(np.ones((m, k), np.uint16)))
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+
+
 @pytest.mark.parametrize("wl", [W.TINY, W.DECODE, W.PREFILL, W.FUSED_QKVG], ids=lambda w: w.name)
 def test_quantize_workload_activations(nv, wl):
     _compare(nv, wl.x())
