@@ -256,6 +256,12 @@ nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream);
  * memory and return.  Values below 1000 are raised to 1000. */
 void nvfp4_set_wait_timeout_ns(uint64_t ns);
 
+/* Number of kernel launches this library has enqueued in this process so far
+ * (every entry point, every device).  Instrumentation for callers that count
+ * device work, e.g. the launches recorded into a CUDA graph; the paper has no
+ * counterpart. */
+uint64_t nvfp4_launch_count(void);
+
 /* Library version string. */
 const char *nvfp4_version(void);
 

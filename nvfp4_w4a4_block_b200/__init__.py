@@ -46,7 +46,7 @@ MAX_SEGMENTS = 8
 EXPORTED = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize_act",
             "nvfp4_pack_weight", "nvfp4_gemm", "nvfp4_linear", "nvfp4_linear_fused", "nvfp4_get_device_error",
             "nvfp4_set_wait_timeout_ns", "nvfp4_version", "nvfp4_linear_fused_noalloc", "nvfp4_dequantize",
-            "nvfp4_import_weight_scales", "nvfp4_harmonize_scales")
+            "nvfp4_import_weight_scales", "nvfp4_harmonize_scales", "nvfp4_launch_count")
 
 
 class NVFP4Error(RuntimeError):
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
                 L.nvfp4_sf_bytes.argtypes, L.nvfp4_sf_bytes.restype = [i64, i64], sz
                 L.nvfp4_workspace_bytes.argtypes, L.nvfp4_workspace_bytes.restype = [i64, i64, i64], sz
                 L.nvfp4_set_wait_timeout_ns.argtypes, L.nvfp4_set_wait_timeout_ns.restype = [ctypes.c_uint64], None
+                L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
                 L.nvfp4_get_device_error.argtypes, L.nvfp4_get_device_error.restype = [vp], ci
                 L.nvfp4_quantize_act.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, sz, vp]
                 L.nvfp4_quantize_act.restype = ci
@@ -115,6 +116,11 @@ def sf_bytes(rows: int, k: int) -> int:
 
 def workspace_bytes(m: int, n: int, k: int) -> int:
     return int(lib().nvfp4_workspace_bytes(m, n, k))
+
+
+def launch_count() -> int:
+    """Kernel launches this library has enqueued in this process so far."""
+    return int(lib().nvfp4_launch_count())
 
 
 def set_wait_timeout_ns(ns: int):

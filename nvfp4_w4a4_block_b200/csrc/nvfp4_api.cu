@@ -37,6 +37,7 @@ constexpr int kMaxPartials = 1024;
 constexpr size_t kAlign = 256;
 
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+std::atomic<uint64_t> g_launches{0};       // kernel launches enqueued by this library (process-wide)
 std::atomic<int> g_use_pair_kernel{1};   // prefill GEMM on CTA pairs (else one CTA per 128 x 256 tile)
 
 struct DeviceInfo {
@@ -80,7 +81,10 @@ cudaError_t launch(void (*kernel)(KArgs...), int grid, int block, size_t smem, c
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e == cudaSuccess)
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e;
 }
 
 // One-time per-device set-up: capability check, SM count, kernel attributes,
@@ -534,6 +538,8 @@ size_t nvfp4_workspace_bytes(int64_t m, int64_t n, int64_t k)
 }
 
 void nvfp4_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns < 1000 ? 1000 : ns); }
+
+uint64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 nvfp4_status nvfp4_quantize_act(const void *x, int64_t m, int64_t k, int64_t ldx, const float *gscale_in,
                                 float *gscale_out, uint8_t *q, uint8_t *sf, void *workspace, size_t ws_bytes,
