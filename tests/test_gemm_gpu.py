@@ -176,6 +176,24 @@ def test_layer_equals_quantize_then_gemm(nv, m, static):
         assert torch.equal(fused, split)
 
 
+@pytest.mark.parametrize("m", [8, 40, 300])
+def test_strided_output_rows_leave_the_gap_untouched(nv, m):
+    """Y with a row stride beyond N (the bf16 tile stores go through TMA with
+    the caller's stride): the N columns match the contiguous result bit for bit
+    and the padding columns keep their contents."""
+    import torch
+    n, k = 328, 640
+    xb, wb, off = W.random_case(12, m, n, k, seg_rows=[136, 192])
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    ref = nv.linear_fused(x, pw)
+    big = torch.full((m, n + 72), 3.0, dtype=torch.bfloat16, device="cuda")
+    nv.linear_fused(x, pw, out=big[:, :n])
+    torch.cuda.synchronize()
+    assert torch.equal(big[:, :n], ref)
+    assert (big[:, n:] == 3.0).all()
+
+
 def test_static_activation_scale(nv):
     xb, wb, off = W.random_case(11, 140, 256, 640)
     y, ref, _ = _layer(nv, xb, wb, off, act_static=0.004, flags=nv.FLAG_F32_OUT)
