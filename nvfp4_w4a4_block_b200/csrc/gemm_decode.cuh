@@ -1,6 +1,6 @@
 // gemm_decode.cuh -- block-scaled FP4 GEMM for few tokens (M <= 64), sm_100a.
 //
-// Same product and epilogue as gemm_sm100.cuh ("Why Gated DeltaNet Survives 4-Bit
+// Same product and epilogue as gemm_pair.cuh ("Why Gated DeltaNet Survives 4-Bit
 // Quantization", §2 "NVFP4"; per-module global scales of §6), organised for the
 // decode regime, which that paper calls weight-bandwidth-bound (§4) and where it
 // attributes the remaining loss to small-batch activation quantization (§9):

@@ -1,9 +1,12 @@
 // gemm_pair.cuh -- block-scaled FP4 GEMM on CTA pairs (tcgen05 cta_group::2), sm_100a.
 //
-// Same product and epilogue as gemm_sm100.cuh ("Why Gated DeltaNet Survives 4-Bit
-// Quantization", §2 "NVFP4": the GEMM runs on native 4-bit tensor cores; §6:
-// per-module global scales of a fused GEMM stay separate), organised for the
-// compute-bound prefill regime:
+// Computes Y[m, n] = alpha[n] * sum_k (e2m1(Qx[m,k]) * e4m3(SFx[m,k/16])) *
+//                                     (e2m1(Qw[n,k]) * e4m3(SFw[n,k/16]))
+// with FP32 accumulation in tensor memory and alpha[n] = s_x * s_w[segment(n)]:
+// the W4A4 GEMM of "Why Gated DeltaNet Survives 4-Bit Quantization" (§2 "NVFP4":
+// the GEMM runs on native 4-bit tensor cores) with the per-module global scales
+// of a fused GEMM kept apart (§6 "Per-module calibration vs. fused-GEMM
+// scaling").  Organised for the compute-bound prefill regime:
 //
 //   * Two CTAs on neighbouring SMs (a cluster of 2) own a 256 x 256 output tile.
 //     The even CTA issues one M=256, N=256, K=64 block-scaled MMA per 64-deep K

@@ -20,7 +20,6 @@
 #include "convert.cuh"
 #include "gemm_decode.cuh"
 #include "gemm_pair.cuh"
-#include "gemm_sm100.cuh"
 #include "quantize.cuh"
 
 // Device scratch of nvfp4_linear_fused_noalloc (see include/nvfp4.h).  In host
@@ -38,7 +37,6 @@ constexpr size_t kAlign = 256;
 
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 std::atomic<uint64_t> g_launches{0};       // kernel launches enqueued by this library (process-wide)
-std::atomic<int> g_use_pair_kernel{1};   // prefill GEMM on CTA pairs (else one CTA per 128 x 256 tile)
 
 struct DeviceInfo {
     bool ready = false;
@@ -107,9 +105,7 @@ nvfp4_status device_setup(int *sms)
             d.status = NVFP4_ERR_UNSUPPORTED_DEVICE;
             return d.status;
         }
-        if (cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(pair::nvfp4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(pair::nvfp4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  pair::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Cfg<8>::SMEM_ALLOC) != cudaSuccess ||
@@ -406,7 +402,7 @@ nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s
 }
 
 // GEMM + epilogue.  Up to 64 tokens take the swapped decode kernel, more take
-// the persistent 128 x 256 tile kernel.  `pdl` is set only when the preceding
+// the persistent CTA-pair kernel (256 x 256 tiles).  `pdl` is set only when the preceding
 // kernel in the stream is this library's quantizer, whose early trigger comes
 // after all earlier work has completed (the decode kernel reads weights before
 // it waits on that quantizer).
@@ -423,39 +419,7 @@ nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x
         return launch_decode<32>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
     if (m <= 64)
         return launch_decode<64>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
-    if (g_use_pair_kernel)
-        return launch_pair(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, sms, pdl,
-                           stream);
-    CUtensorMap ta, tb;
-    nvfp4_status st = make_map(&ta, qx, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(m), gemm::BM);
-    if (st != NVFP4_OK)
-        return st;
-    st = make_map(&tb, qw, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n), gemm::BN);
-    if (st != NVFP4_OK)
-        return st;
-    gemm::Params p;
-    memset(&p, 0, sizeof p);
-    p.sfa = sfx;
-    p.sfb = sfw;
-    p.m = static_cast<int>(m);
-    p.n = static_cast<int>(n);
-    p.k = static_cast<int>(k);
-    p.tiles_m = static_cast<int>((m + gemm::BM - 1) / gemm::BM);
-    p.tiles_n = static_cast<int>((n + gemm::BN - 1) / gemm::BN);
-    p.atoms_k = k / 64;
-    p.k_stages = static_cast<int>((k + gemm::BK - 1) / gemm::BK);
-    p.y = y;
-    p.ldy = ldy;
-    p.s_x = s_x;
-    p.s_w = seg_gscales;
-    p.nseg = nseg;
-    for (int s = 0; s < nseg; ++s)
-        p.seg_end[s] = static_cast<int>(seg_ends[s]);
-    p.flags = flags;
-    p.timeout_ns = g_timeout_ns.load();
-    const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    return cuda_status(launch(gemm::nvfp4_gemm_kernel, grid, gemm::THREADS, gemm::SMEM_ALLOC, stream, pdl, ta, tb, p));
+    return launch_pair(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, sms, pdl, stream);
 }
 
 struct WorkspaceLayout {
