@@ -757,6 +757,7 @@ PROFILE_CASES = {
     "quantize_32768x17408_static": lambda L: _prof_quantize(32768, 17408, L, True),
     "quantize_32768x17408_dynamic": lambda L: _prof_quantize(32768, 17408, L, False),
     "decode_call_m32": lambda L: _prof_decode_call(32, L),
+    "decode_call_m8": lambda L: _prof_decode_call(8, L),
     "dequantize_34816x5120": lambda L: _prof_convert("dequantize", L),
     "import_scales_34816x5120": lambda L: _prof_convert("import", L),
     "harmonize_34816x5120": lambda L: _prof_convert("harmonize", L),

@@ -352,13 +352,27 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     const int64_t total = p.rows * upr;
     const int64_t nthreads = static_cast<int64_t>(kClusterCtas) * kClusterThreads;
     const int64_t gtid = static_cast<int64_t>(cta_rank_in_cluster()) * kClusterThreads + threadIdx.x;
+    // Unit j of this thread is gtid + j * nthreads; its (row, column) advance by a
+    // fixed step, so only the first needs a division.
+    const int64_t step_r = nthreads / upr, step_c = nthreads % upr;
+    int64_t row[kClusterUnits], col[kClusterUnits];
+    row[0] = gtid / upr;
+    col[0] = gtid % upr;
+#pragma unroll
+    for (int j = 1; j < kClusterUnits; ++j) {
+        row[j] = row[j - 1] + step_r;
+        col[j] = col[j - 1] + step_c;
+        if (col[j] >= upr) {
+            col[j] -= upr;
+            ++row[j];
+        }
+    }
     uint4 v[kClusterUnits];
     uint32_t b = 0;
 #pragma unroll
     for (int j = 0; j < kClusterUnits; ++j) {
-        const int64_t u = gtid + j * nthreads;
-        v[j] = u < total ? __ldg(reinterpret_cast<const uint4 *>(p.x + (u / upr) * p.ldx + (u % upr) * 8))
-                         : make_uint4(0, 0, 0, 0);
+        v[j] = row[j] < p.rows ? __ldg(reinterpret_cast<const uint4 *>(p.x + row[j] * p.ldx + col[j] * 8))
+                               : make_uint4(0, 0, 0, 0);
         b = max(b, absmax_bits8(v[j]));
     }
 #pragma unroll
@@ -400,8 +414,8 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
         if (__shfl_sync(0xFFFFFFFFu, u, 0) >= total)       // warp-uniform: lane 0 holds the warp's first unit
             break;
         const bool active = u < total;
-        const int64_t r_ = active ? u / upr : 0;
-        const int64_t c8 = active ? u % upr : 0;
+        const int64_t r_ = active ? row[j] : 0;
+        const int64_t c8 = active ? col[j] : 0;
         uint32_t bm = absmax_bits8(v[j]);
         bm = max(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
         const float bmax = __uint_as_float(bm << 16);
