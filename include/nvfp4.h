@@ -85,6 +85,11 @@ typedef enum {
 #define NVFP4_FLAG_F32_OUT 0x1u              /* write fp32 instead of bf16 (numerics checks) */
 #define NVFP4_FLAG_COLLAPSED_MAX_SCALE 0x2u  /* negative control: every column uses s_x * max(s_w),
                                                 the mismatch of the paper's §6; never for serving */
+#define NVFP4_FLAG_TEST_STALL 0x100u         /* testing only: the GEMM's producer withholds its second
+                                                K stage, so a bounded pipeline wait runs out; the call
+                                                writes no valid output and records NVFP4_ERR_TIMEOUT in
+                                                the device error word (pair it with a short
+                                                nvfp4_set_wait_timeout_ns).  No paper counterpart. */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *nvfp4_status_string(nvfp4_status st);

@@ -41,6 +41,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 FLAG_F32_OUT = 0x1
 FLAG_COLLAPSED_MAX_SCALE = 0x2
+FLAG_TEST_STALL = 0x100
 MAX_SEGMENTS = 8
 
 EXPORTED = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize_act",

@@ -77,6 +77,7 @@ struct Params {
     int seg_end[8];
     unsigned flags;
     uint64_t timeout_ns;
+    int stall_stage;             // testing: K stage whose loads are withheld (-1: none)
 };
 
 template <int T>
@@ -128,7 +129,9 @@ __global__ void __launch_bounds__(THREADS, 2)
         for (int ks = 0; ks < pre; ++ks) {
             const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
             const uint8_t *sfw_src = p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512;
-            if (elect_one()) {
+            // Testing hook: withholding one stage (no arrival, no copies) makes the
+            // MMA issuer's bounded wait on it run out.
+            if (ks != p.stall_stage && elect_one()) {
                 mbar_arrive_expect_tx(&full[ks], A_BYTES + C::B_BYTES + 2 * nkb * 512);
                 tma_load_2d(smem + C::OFF_A + ks * A_BYTES, &tm_w, ks * (BK / 2), w0, &full[ks]);
                 bulk_load(smem + C::OFF_SFA + ks * SF_BYTES, sfw_src, nkb * 512, &full[ks]);
@@ -138,7 +141,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         pdl_wait_prerequisites();                // activation codes/scales are now written
         for (int ks = 0; ks < pre; ++ks) {
             const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
-            if (elect_one()) {
+            if (ks != p.stall_stage && elect_one()) {
                 tma_load_2d(smem + C::OFF_B + ks * C::B_BYTES, &tm_x, ks * (BK / 2), 0, &full[ks]);
                 bulk_load(smem + C::OFF_SFB + ks * SF_BYTES, p.sfx + static_cast<int64_t>(ks * KB) * 512, nkb * 512,
                           &full[ks]);
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                 break;
             const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
             const uint8_t *sfw_src = p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512;
-            if (elect_one()) {
+            if (ks != p.stall_stage && elect_one()) {
                 mbar_arrive_expect_tx(&full[stage], A_BYTES + C::B_BYTES + 2 * nkb * 512);
                 tma_load_2d(smem + C::OFF_A + stage * A_BYTES, &tm_w, ks * (BK / 2), w0, &full[stage]);
                 bulk_load(smem + C::OFF_SFA + stage * SF_BYTES, sfw_src, nkb * 512, &full[stage]);
@@ -172,6 +175,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         // min(STAGES, issued) issues are the only ones possibly in flight.
         for (int j = 0; j < min(C::STAGES, issued); ++j) {
             const int ks = issued - 1 - j;
+            if (ks == p.stall_stage)
+                continue;                        // withheld: nothing in flight
             const int s = ks % C::STAGES;
             const uint32_t ph = static_cast<uint32_t>((ks / C::STAGES) & 1);
             volatile int no_abort = 0;

@@ -80,6 +80,7 @@ struct Params {
     int seg_end[8];
     unsigned flags;
     uint64_t timeout_ns;
+    int stall_stage;             // testing: K stage of each pair's first tile whose loads are withheld (-1: none)
 };
 
 // Segment (module) of output column `col`.
@@ -174,7 +175,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (!ok)
                     break;
                 const uint32_t bar = bar0 + stage * 8;
-                if (elect_one()) {
+                // Testing hook: withholding one stage (no arrival, no copies) makes the
+                // MMA issuer's bounded wait on it run out.
+                const bool withhold = tile == pair_id && ks == p.stall_stage;
+                if (!withhold && elect_one()) {
                     if (rank == 0)
                         mbar_arrive_expect_tx(&full[stage], TX_BYTES);
                     tma_load_2d_pair_hint(smem + OFF_A + stage * A_BYTES, &tm_a, ks * (BK / 2), row_a, bar, keep);
@@ -382,6 +386,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // A role gave up: copies it or another role issued may still be landing
+        // (their barriers are no longer waited on).  Give them time before the
+        // shared memory and tensor memory are released.
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 100000ull) {
+        }
+    }
     __syncwarp();
     cluster_sync_all();                                 // the peer's MMAs and copies are finished
     if (threadIdx.x == 0 && *abort_flag)

@@ -124,6 +124,11 @@ nvfp4_status device_setup(int *sms)
                 return NVFP4_ERR_CUDA;
             g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
         }
+        // The decode-size quantizer runs as one cluster of 16 CTAs (beyond the
+        // portable 8, which sm_100 allows once the kernel opts in).
+        if (cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
         int occ = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_tile_kernel, kQuantThreads, 0) !=
             cudaSuccess)
@@ -205,7 +210,7 @@ int quant_grid(int sms, int64_t rows, int64_t k)
 }
 
 // Quantization of [rows, k] (rows split into segments).  One segment, dynamic
-// scale, at most 65536 elements (decode): one cluster launch reduces the amax
+// scale, at most 196608 elements (decode): one cluster launch reduces the amax
 // and encodes.  Up to 2^20 elements: the per-unit encoder, after an amax pass in
 // dynamic mode.  Larger (or several segments): amax passes and the tiled encoder.
 nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx, const int64_t *seg_ends, int nseg,
@@ -359,6 +364,7 @@ nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x
         p.seg_end[s] = static_cast<int>(seg_ends[s]);
     p.flags = flags;
     p.timeout_ns = g_timeout_ns.load();
+    p.stall_stage = (flags & NVFP4_FLAG_TEST_STALL) ? 1 : -1;
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
     return cuda_status(launch(pair::nvfp4_gemm_pair_kernel, static_cast<int>(2 * pairs), pair::THREADS,
@@ -396,6 +402,7 @@ nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s
         p.seg_end[s] = static_cast<int>(seg_ends[s]);
     p.flags = flags;
     p.timeout_ns = g_timeout_ns.load();
+    p.stall_stage = (flags & NVFP4_FLAG_TEST_STALL) ? 1 : -1;
     const int grid = static_cast<int>((n + decode::BW - 1) / decode::BW);
     return cuda_status(launch(decode::nvfp4_gemm_decode_kernel<T>, grid, decode::THREADS, decode::Cfg<T>::SMEM_ALLOC,
                               stream, pdl, tw, tx, p));
@@ -442,7 +449,7 @@ nvfp4_status check_gemm_args(const uint8_t *qx, const uint8_t *sfx, const float 
 {
     if (m < 0 || n <= 0 || k <= 0)
         return NVFP4_ERR_INVALID_ARG;
-    if (flags & ~(NVFP4_FLAG_F32_OUT | NVFP4_FLAG_COLLAPSED_MAX_SCALE))
+    if (flags & ~(NVFP4_FLAG_F32_OUT | NVFP4_FLAG_COLLAPSED_MAX_SCALE | NVFP4_FLAG_TEST_STALL))
         return NVFP4_ERR_INVALID_ARG;
     if (k % 64 != 0 || n % 8 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;

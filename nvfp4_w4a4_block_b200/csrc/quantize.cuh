@@ -308,14 +308,14 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
 // ------------------------------------------------------------------ encode, one cluster
 
 // Decode-sized activations in dynamic mode, in one launch: a cluster of
-// kClusterCtas CTAs holds the whole tensor in registers (at most
+// kClusterCtas CTAs (16: a non-portable cluster size the launcher opts into) holds the whole tensor in registers (at most
 // kClusterUnits 16-byte units per thread), reduces the absolute maximum over
 // the cluster through distributed shared memory, and encodes from the same
 // registers -- one read of X, no amax pass, no workspace.  Unit-to-lane mapping,
 // arithmetic and stores are those of quantize_kernel.
-constexpr int kClusterCtas = 8;
+constexpr int kClusterCtas = 16;
 constexpr int kClusterThreads = 512;
-constexpr int kClusterUnits = 2;
+constexpr int kClusterUnits = 3;
 
 __device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr)
 {

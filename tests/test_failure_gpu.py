@@ -1,0 +1,50 @@
+"""Failure detection on the GPU without a fault: the GEMM's pipeline waits are
+bounded, and a wait that runs out is reported through the device error word
+while the context stays usable.  The stall comes from a testing flag with which
+the producer withholds one K stage (nothing is in flight for it), so the MMA
+issuer's bounded wait runs out; every other role then gives up on its own
+bounded waits, drains what it issued and frees its tensor memory."""
+import numpy as np
+import pytest
+
+import oracle
+from nvfp4_w4a4_block_b200 import workloads as W
+
+from _helpers import assert_gemm_close, to_cuda_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import nvfp4_w4a4_block_b200 as nv
+    nv.lib()
+    return nv
+
+
+@pytest.mark.parametrize("m", [8, 40, 300], ids=["decode_T8", "decode_T64", "pair"])
+def test_gemm_wait_timeout_is_reported_and_the_context_stays_usable(nv, m):
+    import torch
+    n, k = 392, 1344
+    xb, wb, off = W.random_case(70 + m, m, n, k, seg_rows=[128, 264])
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    qx, sfx, sx = nv.quantize_act(x)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    nv.set_wait_timeout_ns(2_000_000)                  # 2 ms per wait
+    try:
+        nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT | nv.FLAG_TEST_STALL)
+        assert nv.get_device_error() == nv.ERR_TIMEOUT
+        assert nv.get_device_error() == nv.OK          # read and cleared
+    finally:
+        nv.set_wait_timeout_ns(2_000_000_000)
+    # The same context computes the right answer afterwards.
+    y = nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    ref = oracle.linear_reference(xb, wb, off)
+    assert_gemm_close(y.cpu().numpy(), ref["y"], bf16=False)
