@@ -60,6 +60,9 @@ def _load():
         lib.or_bf16_from_f64.argtypes, lib.or_bf16_from_f64.restype = [f64], ctypes.c_uint16
         lib.or_dequantize_bf16.argtypes, lib.or_dequantize_bf16.restype = [vp, vp, i64, i64, vp, vp], None
         lib.or_harmonize.argtypes, lib.or_harmonize.restype = [vp, i64, i64, vp, ctypes.c_int, vp], f32
+        lib.or_e2m1_encode_patterns.argtypes = [ctypes.c_uint64, ctypes.c_uint64, vp]
+        lib.or_e2m1_encode_patterns.restype = None
+        lib.or_e4m3_encode_patterns.argtypes, lib.or_e4m3_encode_patterns.restype = [vp, i64, vp], None
         _lib = lib
     return _lib
 
@@ -85,6 +88,21 @@ def e2m1_encode(v: float) -> int:
 
 def e4m3_encode(v: float) -> int:
     return int(_load().or_e4m3_encode(float(v)))
+
+
+def e2m1_encode_patterns(start: int, count: int) -> np.ndarray:
+    """E2M1 codes of the fp32 bit patterns start .. start+count-1 (one byte each)."""
+    out = np.empty(count, dtype=np.uint8)
+    _load().or_e2m1_encode_patterns(start, count, _ptr(out))
+    return out
+
+
+def e4m3_encode_patterns(pats: np.ndarray) -> np.ndarray:
+    """E4M3 codes of the given fp32 bit patterns."""
+    pats = np.ascontiguousarray(pats, dtype=np.uint32)
+    out = np.empty(pats.size, dtype=np.uint8)
+    _load().or_e4m3_encode_patterns(_ptr(pats), pats.size, _ptr(out))
+    return out
 
 
 def num_threads() -> int:

@@ -396,3 +396,30 @@ float or_harmonize(uint8_t *sf, int64_t rows, int64_t k, const int64_t *seg_offs
     return shared;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Bulk encodes for comparisons over whole ranges of fp32 bit patterns      */
+/* ------------------------------------------------------------------------ */
+
+/* out[i] = E2M1 code (R7) of the fp32 whose bit pattern is start + i. */
+void or_e2m1_encode_patterns(uint64_t start, uint64_t count, uint8_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < (int64_t)count; ++i) {
+        uint32_t u = (uint32_t)(start + (uint64_t)i);
+        float v;
+        memcpy(&v, &u, sizeof v);
+        out[i] = (uint8_t)or_e2m1_encode(v);
+    }
+}
+
+/* out[i] = E4M3 code (R5) of the fp32 whose bit pattern is pats[i]. */
+void or_e4m3_encode_patterns(const uint32_t *pats, int64_t count, uint8_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) {
+        float v;
+        memcpy(&v, &pats[i], sizeof v);
+        out[i] = (uint8_t)or_e4m3_encode(v);
+    }
+}
+
