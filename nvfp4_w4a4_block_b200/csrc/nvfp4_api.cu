@@ -247,6 +247,7 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
         qp.partial = partials;
         qp.npartial = ga;
         qp.scale_out = scale_out;
+        qp.timeout_ns = g_timeout_ns.load();
         if (cluster)
             return cuda_status(launch(quantize_cluster_kernel, kClusterCtas, kClusterThreads, 0, stream, true, qp));
         const int grid = quant_grid(sms, rows, k);

@@ -168,6 +168,7 @@ struct QuantParams {
     const uint32_t *partial;     // [nseg][npartial] amax partials (dynamic)
     int npartial;
     float *scale_out;            // [nseg]
+    uint64_t timeout_ns;         // bound on the cluster kernel's wait for its peers' maxima
 };
 
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
@@ -317,33 +318,31 @@ constexpr int kClusterCtas = 16;
 constexpr int kClusterThreads = 512;
 constexpr int kClusterUnits = 3;
 
-__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr)
-{
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ uint32_t cta_rank_in_cluster()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_barrier()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
     quantize_cluster_kernel(QuantParams p)
 {
     __shared__ uint32_t s_red[kClusterThreads / 32];
-    __shared__ uint32_t s_cta_max;
+    __shared__ uint32_t s_peer_max[kClusterCtas];        // entry r: CTA r's maximum, pushed by CTA r
+    __shared__ __align__(8) uint64_t s_pushes;           // completes when all kClusterCtas entries landed
     __shared__ float s_sc[2];
+    __shared__ int s_abort;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+
+    // The exchange of CTA maxima: every CTA stores its maximum into entry `rank`
+    // of every CTA's s_peer_max (itself included) with st.async, whose bytes
+    // complete the receiver's s_pushes.  A cluster barrier phase (arrive here,
+    // wait just before the first push) orders each barrier's initialisation
+    // before any push; its latency hides under the loads.  A second phase
+    // (arrive once the pushes to this CTA have landed, wait at the very end)
+    // keeps every CTA resident until its own pushes have been received.
+    if (threadIdx.x == 0) {
+        mbar_init(&s_pushes, 1);
+        s_abort = 0;
+        fence_barrier_init();
+        mbar_arrive_expect_tx(&s_pushes, 4u * kClusterCtas);
+    }
+    cluster_arrive_release();
 
     pdl_wait_prerequisites();
     pdl_launch_dependents();
@@ -351,7 +350,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     const int64_t upr = p.k >> 3;
     const int64_t total = p.rows * upr;
     const int64_t nthreads = static_cast<int64_t>(kClusterCtas) * kClusterThreads;
-    const int64_t gtid = static_cast<int64_t>(cta_rank_in_cluster()) * kClusterThreads + threadIdx.x;
+    const int64_t gtid = static_cast<int64_t>(rank) * kClusterThreads + threadIdx.x;
     // Unit j of this thread is gtid + j * nthreads; its (row, column) advance by a
     // fixed step, so only the first needs a division.
     const int64_t step_r = nthreads / upr, step_c = nthreads % upr;
@@ -381,31 +380,37 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     if (lane == 0)
         s_red[threadIdx.x >> 5] = b;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t m = 0;
-        for (int w = 0; w < kClusterThreads / 32; ++w)
-            m = max(m, s_red[w]);
-        s_cta_max = m;
-    }
-    cluster_barrier();                                   // every CTA's maximum is in its shared memory
-    if (threadIdx.x == 0) {
-        uint32_t m = 0;
-        for (int r = 0; r < kClusterCtas; ++r)
-            m = max(m, ld_shared_cluster_u32(map_to_rank(smem_u32(&s_cta_max), static_cast<uint32_t>(r))));
-        float sv = __fdiv_rn(__uint_as_float(m << 16), 2688.0f);
-        if (m >= 0x7F80u) {
-            if (cta_rank_in_cluster() == 0)
-                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
-            sv = 0.0f;
+    cluster_wait_acquire();                              // every CTA's s_pushes is initialised
+    if (threadIdx.x < 32) {
+        uint32_t m = lane < kClusterThreads / 32 ? s_red[lane] : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane < kClusterCtas)
+            st_async_remote_u32(map_to_rank(smem_u32(&s_peer_max[rank]), static_cast<uint32_t>(lane)), m,
+                                map_to_rank(smem_u32(&s_pushes), static_cast<uint32_t>(lane)));
+        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&s_pushes, 0, &s_abort, p.timeout_ns));
+        if (lane == 0) {
+            uint32_t g = 0;
+            for (int r = 0; r < kClusterCtas; ++r)
+                g = max(g, s_peer_max[r]);
+            float sv = __fdiv_rn(__uint_as_float(g << 16), 2688.0f);
+            if (!ok) {
+                raise_device_error(6u /* NVFP4_ERR_TIMEOUT */);
+                sv = 0.0f;
+            } else if (g >= 0x7F80u) {
+                if (rank == 0)
+                    raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
+                sv = 0.0f;
+            }
+            s_sc[0] = sv;
+            s_sc[1] = __fmul_rn(sv, 6.0f);
+            if (rank == 0)
+                p.scale_out[0] = sv;
         }
-        s_sc[0] = sv;
-        s_sc[1] = __fmul_rn(sv, 6.0f);
-        if (cta_rank_in_cluster() == 0)
-            p.scale_out[0] = sv;
     }
-    // The peers' maxima have been read: no CTA of the cluster touches another's
-    // shared memory after this barrier, so each may run to its end.
-    cluster_barrier();
+    __syncthreads();
+    cluster_arrive_relaxed();                            // the pushes to this CTA have landed
     const float s = s_sc[0], dg = s_sc[1];
 
 #pragma unroll
@@ -445,6 +450,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
         const int64_t kb = (i % (p.kb_pad >> 2)) << 2;
         *reinterpret_cast<uint32_t *>(p.sf + sf_atom_offset(row, kb, p.kb_pad)) = 0u;
     }
+    cluster_wait_acquire();                              // every push from this CTA has been received
 }
 
 // ------------------------------------------------------------------ encode, tiled

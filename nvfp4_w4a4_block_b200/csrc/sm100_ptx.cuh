@@ -348,6 +348,32 @@ __device__ __forceinline__ void cluster_sync_all()
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// The two halves of a cluster barrier phase, for callers that overlap other
+// work with the barrier's latency.  Every thread of every CTA takes part.
+__device__ __forceinline__ void cluster_arrive_release()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_acquire()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Stores a word into the shared memory of a CTA of the cluster and counts its
+// 4 bytes on that CTA's mbarrier (both addresses from map_to_rank).
+__device__ __forceinline__ void st_async_remote_u32(uint32_t cluster_addr, uint32_t value, uint32_t cluster_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(cluster_addr),
+                 "r"(value), "r"(cluster_bar)
+                 : "memory");
+}
+
 // Arrive on an mbarrier of another CTA of the cluster (address from map_to_rank).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 {
