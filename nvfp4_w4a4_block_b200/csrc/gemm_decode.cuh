@@ -61,6 +61,7 @@ struct Cfg {
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(SMEM_ALLOC <= SMEM_LIMIT, "two CTAs per SM");
     static_assert(B_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+    static_assert(STAGES * A_BYTES >= T * BW * 4, "the epilogue stages a fp32 tile in the weight buffers");
 };
 
 struct Params {
@@ -171,6 +172,10 @@ __global__ void __launch_bounds__(THREADS, 2)
                 phase ^= 1u;
             }
         }
+        // Nothing is left to issue: let the next kernel in the stream be scheduled
+        // into the slots this grid frees (it waits for this grid's completion
+        // before it reads anything this grid writes).
+        pdl_launch_dependents();
         // Every stage issued must have landed before the CTA exits: the last
         // min(STAGES, issued) issues are the only ones possibly in flight.
         for (int j = 0; j < min(C::STAGES, issued); ++j) {
@@ -252,6 +257,11 @@ __global__ void __launch_bounds__(THREADS, 2)
         }
         if (mbar_wait_bounded(acc_full, 0, abort_flag, p.timeout_ns)) {
             tc_fence_after();
+            // Every stage has landed and every MMA has read its operands, so the
+            // stage buffers are free: the tile is staged there as [token][128
+            // columns] and leaves as 16-byte stores along each token's row.
+            const bool f32 = (p.flags & FLAG_F32_OUT) != 0;
+            uint8_t *stg = smem + C::OFF_A;
             constexpr int CH = (T < 32) ? T : 32;
 #pragma unroll
             for (int c0 = 0; c0 < T; c0 += CH) {
@@ -259,22 +269,27 @@ __global__ void __launch_bounds__(THREADS, 2)
                 __syncwarp();
                 tmem_ld_32x32b<CH>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
                 tmem_ld_wait();
-                if (nrow < p.n) {
-                    if (p.flags & FLAG_F32_OUT) {
-                        float *y = reinterpret_cast<float *>(p.y) + nrow;
 #pragma unroll
-                        for (int i = 0; i < CH; ++i)
-                            if (c0 + i < p.m)
-                                y[static_cast<int64_t>(c0 + i) * p.ldy] = __uint_as_float(r[i]) * alpha;
-                    } else {
-                        __nv_bfloat16 *y = reinterpret_cast<__nv_bfloat16 *>(p.y) + nrow;
-#pragma unroll
-                        for (int i = 0; i < CH; ++i)
-                            if (c0 + i < p.m)
-                                y[static_cast<int64_t>(c0 + i) * p.ldy] =
-                                    __float2bfloat16_rn(__uint_as_float(r[i]) * alpha);
-                    }
+                for (int i = 0; i < CH; ++i) {
+                    const float v = __uint_as_float(r[i]) * alpha;
+                    const int e = (c0 + i) * BW + quarter * 32 + lane;
+                    if (f32)
+                        reinterpret_cast<float *>(stg)[e] = v;
+                    else
+                        reinterpret_cast<__nv_bfloat16 *>(stg)[e] = __float2bfloat16_rn(v);
                 }
+            }
+            bar_sync_named(1, 128);                              // the four epilogue warps
+            const int esz = f32 ? 4 : 2;
+            const int row_chunks = BW * esz / 16;                // 16-byte chunks per token row
+            const int rows = min(T, p.m);
+            uint8_t *y = static_cast<uint8_t *>(p.y);
+            for (int idx = static_cast<int>(threadIdx.x) - 64; idx < rows * row_chunks; idx += 128) {
+                const int t = idx / row_chunks, c = idx - t * row_chunks;
+                const int col = w0 + c * (16 / esz);             // n % 8 == 0: a chunk is all in or all out
+                if (col < p.n)
+                    *reinterpret_cast<uint4 *>(y + (static_cast<int64_t>(t) * p.ldy + col) * esz) =
+                        *reinterpret_cast<const uint4 *>(stg + (t * BW) * esz + c * 16);
             }
         }
     }
