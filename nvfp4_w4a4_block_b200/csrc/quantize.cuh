@@ -91,6 +91,26 @@ __device__ __forceinline__ int64_t sf_atom_offset(int64_t row, int64_t kb, int64
     return ((row >> 7) * (kb_pad >> 2) + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
 }
 
+// Zeroes the scale bytes of the pad rows [rows, rows_pad), all of which lie in
+// the last 128-row block.  Thread i of the launch takes the 4-byte word i of
+// that block's atoms (consecutive threads, consecutive words); the word holds
+// row ((i % 128) / 4) + 32 * (i % 4) of its atom.
+__device__ __forceinline__ void zero_pad_scales(uint8_t *sf, int64_t rows, int64_t rows_pad, int64_t kb_pad,
+                                                int64_t gtid, int64_t nthreads)
+{
+    const int64_t last = (rows_pad >> 7) - 1;                  // last 128-row block
+    const int valid = static_cast<int>(rows - last * 128);     // its rows that hold data
+    if (valid >= 128)
+        return;
+    const int64_t atoms = kb_pad >> 2;
+    uint32_t *block = reinterpret_cast<uint32_t *>(sf + last * atoms * 512);
+    for (int64_t i = gtid; i < atoms * 128; i += nthreads) {
+        const int w = static_cast<int>(i & 127);
+        if (((w >> 2) | ((w & 3) << 5)) >= valid)
+            block[i] = 0u;
+    }
+}
+
 // ------------------------------------------------------------------ amax
 
 struct AmaxParams {
@@ -297,13 +317,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
         }
     }
 
-    // Zero the scale bytes of the pad rows [rows, rows_pad): 4 bytes per (row, atom).
-    const int64_t pad_words = (p.rows_pad - p.rows) * (p.kb_pad >> 2);
-    for (int64_t i = gtid; i < pad_words; i += nthreads) {
-        const int64_t row = p.rows + i / (p.kb_pad >> 2);
-        const int64_t kb = (i % (p.kb_pad >> 2)) << 2;
-        *reinterpret_cast<uint32_t *>(p.sf + sf_atom_offset(row, kb, p.kb_pad)) = 0u;
-    }
+    zero_pad_scales(p.sf, p.rows, p.rows_pad, p.kb_pad, gtid, nthreads);
 }
 
 // ------------------------------------------------------------------ encode, one cluster
@@ -443,13 +457,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
                 sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
     }
 
-    // Zero the scale bytes of the pad rows [rows, rows_pad): 4 bytes per (row, atom).
-    const int64_t pad_words = (p.rows_pad - p.rows) * (p.kb_pad >> 2);
-    for (int64_t i = gtid; i < pad_words; i += nthreads) {
-        const int64_t row = p.rows + i / (p.kb_pad >> 2);
-        const int64_t kb = (i % (p.kb_pad >> 2)) << 2;
-        *reinterpret_cast<uint32_t *>(p.sf + sf_atom_offset(row, kb, p.kb_pad)) = 0u;
-    }
+    zero_pad_scales(p.sf, p.rows, p.rows_pad, p.kb_pad, gtid, nthreads);
     cluster_wait_acquire();                              // every push from this CTA has been received
 }
 

@@ -155,17 +155,19 @@ def test_quantize_nonfinite_sets_device_error(nv):
     assert nv.get_device_error() == nv.OK
 
 
-@pytest.mark.parametrize("m,k", [(4, 5120), (8, 5120), (32, 5120), (38, 5120), (39, 5120), (64, 5120),
+@pytest.mark.parametrize("m,k", [(1, 5120), (4, 5120), (8, 5120), (9, 5120), (1, 40960), (1, 41024), (2, 20480),
+                                 (32, 5120), (38, 5120), (39, 5120), (64, 5120),
                                  (11, 17408), (12, 17408), (1, 196608), (1, 196672)])
 def test_quantize_decode_sizes_around_the_one_launch_limit(nv, m, k):
-    """Dynamic-scale activations up to 196608 elements are quantized in one
-    cluster launch (the whole tensor held in registers); just above that the
-    amax pass and the per-unit encoder take over.  Both sides of the limit."""
+    """Dynamic-scale activations are quantized in one launch with the whole
+    tensor held in registers: one CTA up to 40960 elements, one CTA cluster up
+    to 196608; above that the amax pass and the per-unit encoder take over.
+    Both sides of each limit."""
     x, _, _ = W.random_case(33, m, 8, k)
     _compare(nv, x)
 
 
-@pytest.mark.parametrize("m,k", [(8, 5120), (38, 5120)])
+@pytest.mark.parametrize("m,k", [(1, 5120), (8, 5120), (38, 5120)])
 def test_quantize_nonfinite_in_the_one_launch_path(nv, m, k):
     import torch
     x, _, _ = W.random_case(34, m, 8, k)
