@@ -160,12 +160,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ producer (both CTAs)
         // The whole warp walks the schedule (so every operand below is
         // warp-uniform); one elected lane issues the copies.
-        pdl_wait_prerequisites();
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         const uint32_t bar0 = map_to_rank(smem_u32(&full[0]), 0);
         const uint64_t keep = policy_evict_last();       // operand tiles are re-read by other pairs
+        // The weight operand does not depend on the preceding kernel: the weight
+        // tiles and scales of this pair's first `pre` stages are requested before
+        // waiting for it (their slots are free; each stage's barrier expects the
+        // bytes of all four copies of both CTAs).  Testing hook: withholding one
+        // stage (no arrival, no copies) makes the MMA issuer's bounded wait on it
+        // run out.
+        const int pre = pair_id < num_tiles ? min(STAGES, p.k_stages) : 0;
+        {
+            const int nb = pair_id % p.tiles_n;
+            const int row_b = nb * BN + static_cast<int>(rank) * 128;
+            for (int ks = 0; ks < pre; ++ks) {
+                if (ks != p.stall_stage && elect_one()) {
+                    const uint32_t bar = bar0 + ks * 8;
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(&full[ks], TX_BYTES);
+                    tma_load_2d_pair_hint(smem + OFF_B + ks * B_BYTES, &tm_b, ks * (BK / 2), row_b, bar, keep);
+                    tma_load_3d_pair(smem + OFF_SFB + ks * SFB_BYTES, &tm_sfb, 0, ks * KB, nb * 2, bar);
+                }
+                __syncwarp();
+            }
+        }
+        pdl_wait_prerequisites();                        // the activation codes and scales are written
         for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
             const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
             const int row_a = mb * BM + static_cast<int>(rank) * 128;
@@ -175,17 +196,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (!ok)
                     break;
                 const uint32_t bar = bar0 + stage * 8;
-                // Testing hook: withholding one stage (no arrival, no copies) makes the
-                // MMA issuer's bounded wait on it run out.
                 const bool withhold = tile == pair_id && ks == p.stall_stage;
+                const bool weights_issued = tile == pair_id && ks < pre;
                 if (!withhold && elect_one()) {
-                    if (rank == 0)
+                    if (rank == 0 && !weights_issued)
                         mbar_arrive_expect_tx(&full[stage], TX_BYTES);
                     tma_load_2d_pair_hint(smem + OFF_A + stage * A_BYTES, &tm_a, ks * (BK / 2), row_a, bar, keep);
-                    tma_load_2d_pair_hint(smem + OFF_B + stage * B_BYTES, &tm_b, ks * (BK / 2), row_b, bar, keep);
                     tma_load_3d_pair(smem + OFF_SFA + stage * SFA_BYTES, &tm_sfa, 0, ks * KB,
                                      mb * 2 + static_cast<int>(rank), bar);
-                    tma_load_3d_pair(smem + OFF_SFB + stage * SFB_BYTES, &tm_sfb, 0, ks * KB, nb * 2, bar);
+                    if (!weights_issued) {
+                        tma_load_2d_pair_hint(smem + OFF_B + stage * B_BYTES, &tm_b, ks * (BK / 2), row_b, bar, keep);
+                        tma_load_3d_pair(smem + OFF_SFB + stage * SFB_BYTES, &tm_sfb, 0, ks * KB, nb * 2, bar);
+                    }
                 }
                 __syncwarp();
                 if (++stage == STAGES) {
@@ -194,6 +216,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
         }
+        // Nothing is left to issue: let the next kernel in the stream be scheduled
+        // into the slots this grid frees (it waits for this grid's completion
+        // before it reads anything this grid writes).
+        pdl_launch_dependents();
         if (!ok) {
             // Give copies already issued time to land before the CTA can exit.
             const uint64_t t0 = global_timer_ns();
