@@ -51,8 +51,8 @@ DeviceInfo g_dev[64];
 thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
 thread_local int g_expand_ctas = 148;       // resident expansion CTAs on the current device
 constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder below, tiled encoder above
-// Dynamic scale for decode-sized activations: one cluster launch holds the whole
-// tensor in registers (quantize_cluster_kernel) up to this many elements.
+// Decode-sized activations: one cluster launch holds the whole tensor in
+// registers (quantize_cluster_kernel) up to this many elements.
 constexpr int64_t kClusterQuantElems = int64_t(kClusterCtas) * kClusterThreads * kClusterUnits * 8;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -209,8 +209,8 @@ int quant_grid(int sms, int64_t rows, int64_t k)
     return static_cast<int>(g < 1 ? 1 : g);
 }
 
-// Quantization of [rows, k] (rows split into segments).  One segment, dynamic
-// scale, at most 196608 elements (decode): one cluster launch reduces the amax
+// Quantization of [rows, k] (rows split into segments).  One segment, at most
+// 327680 elements (decode): one cluster launch reduces the amax (dynamic scale)
 // and encodes.  Up to 2^20 elements: the per-unit encoder, after an amax pass in
 // dynamic mode.  Larger (or several segments): amax passes and the tiled encoder.
 nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx, const int64_t *seg_ends, int nseg,
@@ -219,7 +219,7 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
 {
     const int ga = amax_grid(sms, rows, k);
     if (nseg == 1 && rows * k <= kSmallQuantElems) {
-        const bool cluster = static_scale == nullptr && rows * k <= kClusterQuantElems;
+        const bool cluster = rows * k <= kClusterQuantElems;
         if (static_scale == nullptr && !cluster) {
             AmaxParams ap;
             ap.x = static_cast<const uint16_t *>(x);

@@ -322,15 +322,16 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
 
 // ------------------------------------------------------------------ encode, one cluster
 
-// Decode-sized activations in dynamic mode, in one launch: a cluster of
-// kClusterCtas CTAs (16: a non-portable cluster size the launcher opts into) holds the whole tensor in registers (at most
-// kClusterUnits 16-byte units per thread), reduces the absolute maximum over
-// the cluster through distributed shared memory, and encodes from the same
-// registers -- one read of X, no amax pass, no workspace.  Unit-to-lane mapping,
-// arithmetic and stores are those of quantize_kernel.
+// Decode-sized activations in one launch: a cluster of kClusterCtas CTAs (16:
+// a non-portable cluster size the launcher opts into) holds the whole tensor in
+// registers (at most kClusterUnits 16-byte units per thread), reduces the
+// absolute maximum over the cluster through distributed shared memory when the
+// scale is dynamic, and encodes from the same registers -- one read of X, no
+// amax pass, no workspace.  Unit-to-lane mapping, arithmetic and stores are
+// those of quantize_kernel.
 constexpr int kClusterCtas = 16;
 constexpr int kClusterThreads = 512;
-constexpr int kClusterUnits = 3;
+constexpr int kClusterUnits = 5;
 
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
     quantize_cluster_kernel(QuantParams p)
@@ -350,13 +351,18 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     // before any push; its latency hides under the loads.  A second phase
     // (arrive once the pushes to this CTA have landed, wait at the very end)
     // keeps every CTA resident until its own pushes have been received.
-    if (threadIdx.x == 0) {
-        mbar_init(&s_pushes, 1);
-        s_abort = 0;
-        fence_barrier_init();
-        mbar_arrive_expect_tx(&s_pushes, 4u * kClusterCtas);
+    // With a given (calibrated) scale there is nothing to exchange: no CTA of
+    // the cluster touches another's shared memory and no barrier phase is used.
+    const bool given = p.static_scale != nullptr;
+    if (!given) {
+        if (threadIdx.x == 0) {
+            mbar_init(&s_pushes, 1);
+            s_abort = 0;
+            fence_barrier_init();
+            mbar_arrive_expect_tx(&s_pushes, 4u * kClusterCtas);
+        }
+        cluster_arrive_release();
     }
-    cluster_arrive_release();
 
     pdl_wait_prerequisites();
     pdl_launch_dependents();
@@ -367,10 +373,12 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     const int64_t gtid = static_cast<int64_t>(rank) * kClusterThreads + threadIdx.x;
     // Unit j of this thread is gtid + j * nthreads; its (row, column) advance by a
     // fixed step, so only the first needs a division.
-    const int64_t step_r = nthreads / upr, step_c = nthreads % upr;
-    int64_t row[kClusterUnits], col[kClusterUnits];
-    row[0] = gtid / upr;
-    col[0] = gtid % upr;
+    // The launch covers at most kClusterCtas * kClusterThreads * kClusterUnits
+    // units, so a unit's row and column fit in 32 bits.
+    const int step_r = static_cast<int>(nthreads / upr), step_c = static_cast<int>(nthreads % upr);
+    int row[kClusterUnits], col[kClusterUnits];
+    row[0] = static_cast<int>(gtid / upr);
+    col[0] = static_cast<int>(gtid % upr);
 #pragma unroll
     for (int j = 1; j < kClusterUnits; ++j) {
         row[j] = row[j - 1] + step_r;
@@ -384,47 +392,62 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     uint32_t b = 0;
 #pragma unroll
     for (int j = 0; j < kClusterUnits; ++j) {
-        v[j] = row[j] < p.rows ? __ldg(reinterpret_cast<const uint4 *>(p.x + row[j] * p.ldx + col[j] * 8))
+        v[j] = row[j] < p.rows ? __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(row[j]) * p.ldx +
+                                                                    col[j] * 8))
                                : make_uint4(0, 0, 0, 0);
         b = max(b, absmax_bits8(v[j]));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
-    if (lane == 0)
-        s_red[threadIdx.x >> 5] = b;
-    __syncthreads();
-    cluster_wait_acquire();                              // every CTA's s_pushes is initialised
-    if (threadIdx.x < 32) {
-        uint32_t m = lane < kClusterThreads / 32 ? s_red[lane] : 0u;
+    if (!given) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        if (lane < kClusterCtas)
-            st_async_remote_u32(map_to_rank(smem_u32(&s_peer_max[rank]), static_cast<uint32_t>(lane)), m,
-                                map_to_rank(smem_u32(&s_pushes), static_cast<uint32_t>(lane)));
-        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&s_pushes, 0, &s_abort, p.timeout_ns));
-        if (lane == 0) {
-            uint32_t g = 0;
-            for (int r = 0; r < kClusterCtas; ++r)
-                g = max(g, s_peer_max[r]);
-            float sv = __fdiv_rn(__uint_as_float(g << 16), 2688.0f);
-            if (!ok) {
-                raise_device_error(6u /* NVFP4_ERR_TIMEOUT */);
-                sv = 0.0f;
-            } else if (g >= 0x7F80u) {
+            b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+        if (lane == 0)
+            s_red[threadIdx.x >> 5] = b;
+        __syncthreads();
+        cluster_wait_acquire();                          // every CTA's s_pushes is initialised
+        if (threadIdx.x < 32) {
+            uint32_t m = lane < kClusterThreads / 32 ? s_red[lane] : 0u;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+            if (lane < kClusterCtas)
+                st_async_remote_u32(map_to_rank(smem_u32(&s_peer_max[rank]), static_cast<uint32_t>(lane)), m,
+                                    map_to_rank(smem_u32(&s_pushes), static_cast<uint32_t>(lane)));
+            const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&s_pushes, 0, &s_abort, p.timeout_ns));
+            if (lane == 0) {
+                uint32_t g = 0;
+                for (int r = 0; r < kClusterCtas; ++r)
+                    g = max(g, s_peer_max[r]);
+                float sv = __fdiv_rn(__uint_as_float(g << 16), 2688.0f);
+                if (!ok) {
+                    raise_device_error(6u /* NVFP4_ERR_TIMEOUT */);
+                    sv = 0.0f;
+                } else if (g >= 0x7F80u) {
+                    if (rank == 0)
+                        raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
+                    sv = 0.0f;
+                }
+                s_sc[0] = sv;
+                s_sc[1] = __fmul_rn(sv, 6.0f);
                 if (rank == 0)
-                    raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
-                sv = 0.0f;
+                    p.scale_out[0] = sv;
             }
-            s_sc[0] = sv;
-            s_sc[1] = __fmul_rn(sv, 6.0f);
-            if (rank == 0)
-                p.scale_out[0] = sv;
         }
+    } else if (threadIdx.x == 0) {
+        float sv = p.static_scale[0];
+        if (!(isfinite(sv) && sv >= 0.0f)) {
+            if (rank == 0)
+                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
+            sv = 0.0f;
+        }
+        s_sc[0] = sv;
+        s_sc[1] = __fmul_rn(sv, 6.0f);
+        if (rank == 0)
+            p.scale_out[0] = sv;
     }
     __syncthreads();
-    cluster_arrive_relaxed();                            // the pushes to this CTA have landed
+    if (!given)
+        cluster_arrive_relaxed();                        // the pushes to this CTA have landed
     const float s = s_sc[0], dg = s_sc[1];
 
 #pragma unroll
@@ -458,7 +481,8 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     }
 
     zero_pad_scales(p.sf, p.rows, p.rows_pad, p.kb_pad, gtid, nthreads);
-    cluster_wait_acquire();                              // every push from this CTA has been received
+    if (!given)
+        cluster_wait_acquire();                          // every push from this CTA has been received
 }
 
 // ------------------------------------------------------------------ encode, tiled

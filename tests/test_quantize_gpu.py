@@ -91,6 +91,25 @@ def test_quantize_static_scale(nv, static):
     _compare(nv, x, static)
 
 
+@pytest.mark.parametrize("bad", [-1.0, float("inf"), float("nan")], ids=["negative", "inf", "nan"])
+@pytest.mark.parametrize("m,k", [(8, 5120), (300, 1088), (1000, 1088)], ids=["cluster", "per_unit", "tiled"])
+def test_quantize_invalid_static_scale_is_reported(nv, m, k, bad):
+    """A given global scale that is negative or not finite is reported as
+    non-finite, and the tensor is encoded as with scale 0 (zero block scales,
+    codes +-0 by sign), on each quantizer path."""
+    import torch
+    x, _, _ = W.random_case(35, m, 8, k)
+    g = torch.tensor([bad], dtype=torch.float32, device="cuda")
+    q, sf, s = nv.quantize_act(to_cuda_bf16(x), gscale=g)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.ERR_NONFINITE
+    assert nv.get_device_error() == nv.OK
+    qo, sfo, _ = _expect(x, 0.0)
+    assert s.item() == 0.0
+    assert np.array_equal(sf.cpu().numpy(), sfo)
+    assert np.array_equal(q.cpu().numpy(), qo)
+
+
 def test_quantize_every_bf16_value_on_identity_scale(nv):
     """Global scale 2^-8 and a 6.0 in every block make the element divisor exactly
     1, so each bf16 value in [-6, 6] is encoded as itself: every tie, every
@@ -157,17 +176,17 @@ def test_quantize_nonfinite_sets_device_error(nv):
 
 @pytest.mark.parametrize("m,k", [(1, 5120), (4, 5120), (8, 5120), (9, 5120), (1, 40960), (1, 41024), (2, 20480),
                                  (32, 5120), (38, 5120), (39, 5120), (64, 5120),
-                                 (11, 17408), (12, 17408), (1, 196608), (1, 196672)])
+                                 (65, 5120), (18, 17408), (19, 17408), (1, 196608), (1, 327680), (1, 327744)])
 def test_quantize_decode_sizes_around_the_one_launch_limit(nv, m, k):
-    """Dynamic-scale activations are quantized in one launch with the whole
-    tensor held in registers: one CTA up to 40960 elements, one CTA cluster up
-    to 196608; above that the amax pass and the per-unit encoder take over.
-    Both sides of each limit."""
+    """Dynamic-scale activations up to 327680 elements are quantized in one
+    cluster launch (the whole tensor held in registers); just above that the
+    amax pass and the per-unit encoder take over.  Both sides of the limit, and
+    shapes whose pad rows fill most of the scale block."""
     x, _, _ = W.random_case(33, m, 8, k)
     _compare(nv, x)
 
 
-@pytest.mark.parametrize("m,k", [(1, 5120), (8, 5120), (38, 5120)])
+@pytest.mark.parametrize("m,k", [(1, 5120), (8, 5120), (38, 5120), (64, 5120)])
 def test_quantize_nonfinite_in_the_one_launch_path(nv, m, k):
     import torch
     x, _, _ = W.random_case(34, m, 8, k)
