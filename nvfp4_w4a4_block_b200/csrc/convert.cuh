@@ -183,17 +183,19 @@ __global__ void __launch_bounds__(kThreads) expand_kernel(ExpandParams p)
         const uint32_t cur[4] = {codes[0], codes[1], codes[2], codes[3]};
         if (t + gridDim.x < tiles)
             load(t + gridDim.x, nrt, nct, sfw, codes);   // next tile's loads in flight during the expansion
+        // The thread's rows in this tile are row0 + 32 j; the segment index only
+        // moves forward along them, and the output pointer advances by 32 rows.
+        const int64_t row0 = rt * 128 + rsub;
+        const int64_t left = row0 >= p.rows ? 0 : (p.rows - row0 + 31) >> 5;   // rows of the thread in this tile
+        const int rows_here = left < 4 ? static_cast<int>(left) : 4;
+        uint16_t *out = p.y + row0 * p.ldy + ct * 64 + g * 8;
+        int seg = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int64_t row = rt * 128 + j * 32 + rsub;
-            if (row >= p.rows)
-                continue;
-            int seg = 0;
-            if (p.nseg > 1) {
-#pragma unroll
-                for (int i = 0; i < kMaxSeg - 1; ++i)
-                    seg += (i + 1 < p.nseg && row >= p.seg_end[i]) ? 1 : 0;
-            }
+            if (j >= rows_here)
+                break;
+            while (seg < p.nseg - 1 && row0 + 32 * j >= p.seg_end[seg])
+                ++seg;
             const uint32_t sb = (sfv[j] >> (8 * (g >> 1))) & 0xFFu;
             const uint4 tv = s_lut[seg * 128 + (sb & 0x7Fu)];
             const BlockTable tb = {tv.x, tv.y, tv.z, tv.w};
@@ -205,7 +207,8 @@ __global__ void __launch_bounds__(kThreads) expand_kernel(ExpandParams p)
             o.y ^= neg;
             o.z ^= neg;
             o.w ^= neg;
-            *reinterpret_cast<uint4 *>(p.y + row * p.ldy + ct * 64 + g * 8) = o;
+            *reinterpret_cast<uint4 *>(out) = o;
+            out += 32 * p.ldy;
         }
         rt = nrt;
         ct = nct;
