@@ -285,7 +285,14 @@ __global__ void __launch_bounds__(kThreads) harmonize_kernel(HarmonizeParams p)
 {
     __shared__ float s_ratio[kMaxSeg];
     __shared__ int s_state;                    // 0 fold, 1 copy unchanged (all zero), 2 bad scale
+    // Per segment, the folded byte of every scale byte b:
+    // E4M3(value(b) * ratio) -- the same fp32 operations as folding it in place.
+    __shared__ uint8_t s_fold[kMaxSeg][256];
+    __shared__ int64_t s_end[kMaxSeg];
     if (threadIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < kMaxSeg; ++i)
+            s_end[i] = p.seg_end[i];
         float shared = 0.0f;
         int bad = 0;
         for (int i = 0; i < p.nseg; ++i) {
@@ -308,30 +315,36 @@ __global__ void __launch_bounds__(kThreads) harmonize_kernel(HarmonizeParams p)
     const int state = s_state;
     if (state == 2)
         return;                                // leave the scales as they are
+    if (state == 0) {
+        for (int idx = threadIdx.x; idx < p.nseg * 256; idx += blockDim.x) {
+            const float folded = __fmul_rn(e4m3_to_f32(static_cast<uint32_t>(idx & 255)), s_ratio[idx >> 8]);
+            s_fold[idx >> 8][idx & 255] = static_cast<uint8_t>(f32_to_e4m3(folded));
+        }
+        __syncthreads();
+    }
+    const int atoms_k = static_cast<int>(p.atoms_k);
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < p.units; u += nthreads) {
         uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.sf_in) + u);
         if (state == 0) {
-            const int64_t rb = (u >> 5) / p.atoms_k;
+            // Word u is line w of atom u / 32: rows 128 rb + 32 j + w (j = 0..3) of
+            // 128-row block rb; the segment index only moves forward along them.
+            const int64_t rb = static_cast<int64_t>(static_cast<uint32_t>(u >> 5) / static_cast<uint32_t>(atoms_k));
             const int w = static_cast<int>(u & 31);
             uint32_t words[4] = {v.x, v.y, v.z, v.w};
+            int seg = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int64_t row = rb * 128 + j * 32 + w;
-                if (row >= p.rows)
-                    continue;                  // pad rows stay as they are
-                int seg = 0;
-#pragma unroll
-                for (int i = 0; i < kMaxSeg - 1; ++i)
-                    seg += (i + 1 < p.nseg && row >= p.seg_end[i]) ? 1 : 0;
-                const float ratio = s_ratio[seg];
-                uint32_t out = 0;
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const float folded = __fmul_rn(e4m3_to_f32((words[j] >> (8 * b)) & 0xFFu), ratio);
-                    out |= f32_to_e4m3(folded) << (8 * b);
+                if (row < p.rows) {            // pad rows stay as they are
+                    while (seg < p.nseg - 1 && row >= s_end[seg])
+                        ++seg;
+                    const uint8_t *f = s_fold[seg];
+                    const uint32_t x = words[j];
+                    words[j] = static_cast<uint32_t>(f[x & 0xFFu]) | (static_cast<uint32_t>(f[(x >> 8) & 0xFFu]) << 8) |
+                               (static_cast<uint32_t>(f[(x >> 16) & 0xFFu]) << 16) |
+                               (static_cast<uint32_t>(f[x >> 24]) << 24);
                 }
-                words[j] = out;
             }
             v = make_uint4(words[0], words[1], words[2], words[3]);
         }
