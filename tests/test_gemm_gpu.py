@@ -74,6 +74,25 @@ def test_gemm_parity_random(nv, m, n, k, segs):
     assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), bf16_rne_from_f32(y32.cpu().numpy()))
 
 
+@pytest.mark.parametrize("m", [8, 40, 200], ids=["decode_T8", "decode_T64", "pair"])
+def test_gemm_eight_modules_some_eight_columns_wide(nv, m):
+    """The largest number of fused modules (eight, each with its own weight
+    global scale, spread 1x-8x), four of them only 8 columns wide -- the finest
+    boundary granularity -- on each GEMM kernel: every output column is scaled by
+    the scale of its own module."""
+    import torch
+    widths = [8, 8, 120, 8, 120, 8, 120, 8]
+    xb, wb, off = W.random_case(71, m, sum(widths), 1088, seg_rows=widths)
+    assert len(off) - 1 == 8
+    y32, ref, pw = _layer(nv, xb, wb, off, flags=nv.FLAG_F32_OUT)
+    assert_gemm_close(y32.cpu().numpy(), ref["y"], bf16=False)
+    g = pw.gscale.cpu().numpy()
+    assert g.max() / g.min() > 4.0                      # a column scaled by another module's scale shows
+    ybf = nv.linear_fused(to_cuda_bf16(xb), pw)
+    torch.cuda.synchronize()
+    assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), bf16_rne_from_f32(y32.cpu().numpy()))
+
+
 @pytest.mark.parametrize("m", [1, 7, 8, 9, 16, 17, 31, 32, 33, 63, 64, 65])
 def test_gemm_token_buckets(nv, m):
     """Every token-count bucket of the swapped decode kernel (8/16/32/64) and the
