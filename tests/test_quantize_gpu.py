@@ -148,15 +148,24 @@ def test_quantize_zero_and_negative_zero(nv):
     _compare(nv, x, 0.5)
 
 
-def test_quantize_strided_rows(nv):
+@pytest.mark.parametrize("m,k,pad", [(64, 256, 128), (8, 5120, 64), (129, 5120, 192), (1000, 1088, 64)],
+                         ids=["cluster_small", "cluster_decode", "per_unit", "tiled"])
+@pytest.mark.parametrize("static", [None, 0.004])
+def test_quantize_strided_rows(nv, m, k, pad, static):
+    """Rows of X further apart than K (a view into a wider buffer, whose extra
+    columns hold large values that must not leak into the amax) on each
+    quantizer path."""
     import torch
-    xb, _, _ = W.random_case(5, 64, 8, 256)
-    big = np.zeros((64, 384), np.uint16)
-    big[:, :256] = xb
-    xt = to_cuda_bf16(big)[:, :256]
-    q, sf, s = nv.quantize_act(xt)
+    xb, _, _ = W.random_case(5, m, 8, k)
+    big = np.full((m, k + pad), W.f32_to_bf16_bits(np.array([1000.0], np.float32))[0], np.uint16)
+    big[:, :k] = xb
+    xt = to_cuda_bf16(big)[:, :k]
+    g = None if static is None else torch.tensor([static], dtype=torch.float32, device="cuda")
+    q, sf, s = nv.quantize_act(xt, gscale=g)
     torch.cuda.synchronize()
-    qo, sfo, so = _expect(xb)
+    assert nv.get_device_error() == nv.OK
+    qo, sfo, so = _expect(xb, static)
+    assert s.item() == float(so)
     assert np.array_equal(q.cpu().numpy(), qo)
     assert np.array_equal(sf.cpu().numpy(), sfo)
 
