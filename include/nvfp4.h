@@ -53,6 +53,12 @@
  * Shape limits: K % 64 == 0, N % 8 == 0, M >= 0 (M == 0 is a no-op),
  * 1 <= nseg <= NVFP4_MAX_SEGMENTS, segment offsets strictly increasing from 0
  * to the segmented extent (N, or the row count), interior offsets multiples of 8.
+ *
+ * Environment: NVFP4_NO_CLUSTER_QUANTIZER=1 (read once per device, at the first
+ * call on it) makes decode-sized activations take the amax pass + per-unit
+ * encoder instead of the one-launch 16-CTA cluster quantizer, as happens anyway
+ * on a device or partition that cannot hold such a cluster.  Results are the
+ * same bytes either way.
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_

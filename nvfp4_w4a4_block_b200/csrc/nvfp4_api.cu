@@ -13,6 +13,7 @@
 #include <atomic>
 #include <cstdint>
 #include <utility>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -44,12 +45,14 @@ struct DeviceInfo {
     int sms = 0;
     int tile_quant_ctas_per_sm = 1;
     int expand_ctas_per_sm = 1;
+    bool cluster_quant = false;     // a 16-CTA cluster of the decode quantizer can be resident
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[64];
 thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
 thread_local int g_expand_ctas = 148;       // resident expansion CTAs on the current device
+thread_local bool g_cluster_quant = false;  // decode quantizer cluster available on the current device
 constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder below, tiled encoder above
 // Decode-sized activations: one cluster launch holds the whole tensor in
 // registers (quantize_cluster_kernel) up to this many elements.
@@ -129,6 +132,22 @@ nvfp4_status device_setup(int *sms)
         if (cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
             cudaSuccess)
             return NVFP4_ERR_CUDA;
+        {
+            // A device (or partition) that cannot hold one such cluster takes the
+            // amax pass + per-unit encoder instead.
+            cudaLaunchConfig_t cc = {};
+            cc.gridDim = dim3(kClusterCtas);
+            cc.blockDim = dim3(kClusterThreads);
+            int nclusters = 0;
+            d.cluster_quant = cudaOccupancyMaxActiveClusters(&nclusters, quantize_cluster_kernel, &cc) == cudaSuccess &&
+                              nclusters >= 1;
+            cudaGetLastError();     // a refused query leaves no sticky error behind
+            // NVFP4_NO_CLUSTER_QUANTIZER=1 takes the same fallback on any device
+            // (it is how the fallback is tested on parts where the cluster fits).
+            const char *no_cluster = std::getenv("NVFP4_NO_CLUSTER_QUANTIZER");
+            if (no_cluster != nullptr && no_cluster[0] == '1')
+                d.cluster_quant = false;
+        }
         int occ = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_tile_kernel, kQuantThreads, 0) !=
             cudaSuccess)
@@ -146,6 +165,7 @@ nvfp4_status device_setup(int *sms)
     *sms = d.sms;
     g_tile_quant_ctas = d.sms * d.tile_quant_ctas_per_sm;
     g_expand_ctas = d.sms * d.expand_ctas_per_sm;
+    g_cluster_quant = d.cluster_quant;
     return d.status;
 }
 
@@ -219,7 +239,7 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
 {
     const int ga = amax_grid(sms, rows, k);
     if (nseg == 1 && rows * k <= kSmallQuantElems) {
-        const bool cluster = rows * k <= kClusterQuantElems;
+        const bool cluster = g_cluster_quant && rows * k <= kClusterQuantElems;
         if (static_scale == nullptr && !cluster) {
             AmaxParams ap;
             ap.x = static_cast<const uint16_t *>(x);

@@ -4,6 +4,8 @@ Codes, scale bytes (physical tensor-core layout, pads included) and the global
 scale must match bit for bit; both sides take every rounding decision in fp32
 with the same operation order.
 """
+import os
+
 import numpy as np
 import pytest
 
@@ -193,6 +195,49 @@ def test_quantize_decode_sizes_around_the_one_launch_limit(nv, m, k):
     shapes whose pad rows fill most of the scale block."""
     x, _, _ = W.random_case(33, m, 8, k)
     _compare(nv, x)
+
+
+def test_fallback_without_the_cluster_quantizer_gives_the_same_bytes(nv):
+    """With the one-launch cluster quantizer switched off (what a device that
+    cannot hold a 16-CTA cluster gets), decode-sized activations take the amax
+    pass and the per-unit encoder: the same codes, scales and global scale, and
+    the same decode layer output.  Runs in a child process, since the choice is
+    made once per device."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, %r); sys.path.insert(0, %r)
+import oracle, nvfp4_w4a4_block_b200 as nv
+from nvfp4_w4a4_block_b200 import workloads as W
+from _helpers import to_cuda_bf16, assert_gemm_close
+nv.lib()
+for m, k, static in [(1, 5120, None), (8, 5120, None), (32, 5120, 0.004), (64, 5120, None)]:
+    x, w, off = W.random_case(36, m, 264, k, seg_rows=[136, 128])
+    g = None if static is None else torch.tensor([static], dtype=torch.float32, device="cuda")
+    xt = to_cuda_bf16(x)
+    c0 = nv.launch_count()
+    q, sf, s = nv.quantize_act(xt, gscale=g)
+    assert nv.launch_count() - c0 == (1 if static is not None else 2)   # encoder (+ amax pass): no cluster
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    so = oracle.global_scale(oracle.amax(x)) if static is None else np.float32(static)
+    qo, sfo = oracle.quantize(x, so)
+    assert np.float32(s.item()).tobytes() == np.float32(so).tobytes()
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_physical(sfo, k))
+    pw = nv.pack_weight(to_cuda_bf16(w), off)
+    y = nv.linear_fused(to_cuda_bf16(x), pw, act_gscale=g, flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+    ref = oracle.linear_reference(x, w, off, act_scale=static)
+    assert_gemm_close(y.cpu().numpy(), ref["y"], bf16=False)
+print("ok")
+""" % (root, os.path.join(root, "tests"))
+    env = dict(os.environ, NVFP4_NO_CLUSTER_QUANTIZER="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.split()[0] == "ok"
 
 
 @pytest.mark.parametrize("m,k", [(1, 5120), (8, 5120), (38, 5120), (64, 5120)])
