@@ -215,12 +215,37 @@ def time_graph(g, reps, per_replay):
     return e0.elapsed_time(e1) / (reps * per_replay)
 
 
+def code_only(text: str) -> str:
+    """C++ source with its comments and blank space removed: what the compiler
+    sees, so that editing a comment does not change a kernel's hash."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] == '"':                     # string literal (PTX text): kept as written
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def kernel_source_hash(files):
-    """Hash of a kernel's own source files (under the package's csrc/)."""
+    """Hash of a kernel's own source files (under the package's csrc/), comments
+    and blank space excluded."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nvfp4_w4a4_block_b200", "csrc")
     for name in files:
-        h.update(open(os.path.join(csrc, name), "rb").read())
+        h.update(code_only(open(os.path.join(csrc, name)).read()).encode())
     return h.hexdigest()[:16]
 
 

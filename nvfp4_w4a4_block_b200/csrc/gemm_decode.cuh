@@ -15,11 +15,13 @@
 //   * The kernel is launched with programmatic stream serialization: the producer
 //     streams the first STAGES weight stages before griddepcontrol.wait, i.e. while
 //     the activation quantizer that precedes it is still running, then loads the
-//     activation stages.
+//     activation stages; once it has issued its last load it lets the next kernel
+//     in the stream be scheduled.
 //
 // Roles: warp 0 producer (TMA + bulk copies), warp 1 MMA issuer (one elected lane),
-// warps 2..5 epilogue (tcgen05.ld of the 128 x T accumulator, x alpha(n), bf16
-// stores of Y[t, n] -- 32 consecutive n per warp per token).
+// warps 2..5 epilogue (tcgen05.ld of the 128 x T accumulator, x alpha(n), the tile
+// staged as [token][128 columns] in the idle stage buffers, then 16-byte stores
+// along each token's row of Y).
 #pragma once
 
 #include <cstdint>

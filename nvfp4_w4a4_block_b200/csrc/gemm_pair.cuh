@@ -16,6 +16,9 @@
 //     for 128 x 256 x 256 MACs, a third less than a single-CTA 128 x 256 tile.
 //   * Five 38 KB stages per CTA.  Both CTAs' TMA loads complete on the even CTA's
 //     stage barrier; the even CTA's tcgen05.commit releases the stage in both.
+//     Launched behind the activation quantizer with programmatic stream
+//     serialization, the producers request the weight tiles and scales of their
+//     first five stages before griddepcontrol.wait.
 //   * Eight epilogue warps per CTA drain the accumulator into registers (128
 //     columns each), hand the tensor memory back to the MMA issuer at once, and
 //     only then scale and convert -- the next tile's MMAs overlap the rest of the
