@@ -75,6 +75,7 @@ constexpr unsigned FLAG_COLLAPSED = 2u;
 struct Params {
     int m, n, k;
     int tiles_m, tiles_n, k_stages;
+    int group_m;                 // tile order: groups of group_m M tiles, N-major inside a group
     void *y;
     int64_t ldy;
     const float *s_x;
@@ -108,6 +109,21 @@ __device__ __forceinline__ void scale32(const Params &p, const float *alpha, int
         for (int i = 0; i < 8; ++i)
             v[8 * g + i] = __uint_as_float(r[8 * g + i]) * a;
     }
+}
+
+// Output tile `tile` of the persistent schedule.  Tiles are visited in groups of
+// group_m consecutive M tiles, N-major inside a group, so that the tiles in
+// flight at once share fewer operand rows and more of them stay in L2.  The
+// producer and the epilogue warps use the same order.
+__device__ __forceinline__ void tile_coords(const Params &p, int tile, int &mb, int &nb)
+{
+    const int group_tiles = p.group_m * p.tiles_n;
+    const int g = tile / group_tiles;
+    const int first_m = g * p.group_m;
+    const int rows = min(p.group_m, p.tiles_m - first_m);
+    const int idx = tile - g * group_tiles;
+    mb = first_m + idx % rows;
+    nb = idx / rows;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
@@ -176,7 +192,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // run out.
         const int pre = pair_id < num_tiles ? min(STAGES, p.k_stages) : 0;
         {
-            const int nb = pair_id % p.tiles_n;
+            int mb0, nb;
+            tile_coords(p, pair_id, mb0, nb);
             const int row_b = nb * BN + static_cast<int>(rank) * 128;
             for (int ks = 0; ks < pre; ++ks) {
                 if (ks != p.stall_stage && elect_one()) {
@@ -191,7 +208,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         pdl_wait_prerequisites();                        // the activation codes and scales are written
         for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
-            const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+            int mb, nb;
+            tile_coords(p, tile, mb, nb);
             const int row_a = mb * BM + static_cast<int>(rank) * 128;
             const int row_b = nb * BN + static_cast<int>(rank) * 128;
             for (int ks = 0; ks < p.k_stages; ++ks) {
@@ -319,7 +337,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint64_t stream_out = policy_evict_first();  // output tiles are written once
         uint32_t acc_phase = 0;
         for (int tile = pair_id; tile < num_tiles; tile += npairs) {
-            const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+            int mb, nb;
+            tile_coords(p, tile, mb, nb);
             const bool ok = mbar_wait_bounded(acc_full, acc_phase, abort_flag, p.timeout_ns);
             // All eight warps take the same decision (each reaches this barrier after
             // its own bounded wait), so the named barriers below cannot strand one.

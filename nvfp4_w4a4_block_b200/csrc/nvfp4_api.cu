@@ -375,6 +375,9 @@ nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x
     p.k = static_cast<int>(k);
     p.tiles_m = static_cast<int>((m + pair::BM - 1) / pair::BM);
     p.tiles_n = static_cast<int>((n + pair::BN - 1) / pair::BN);
+    // Groups of 16 M tiles once there are at least two such groups (measured:
+    // -5% on 8192 x 17408 x 5120; smaller M keeps the plain M-major order).
+    p.group_m = p.tiles_m >= 32 ? 16 : 1;
     p.k_stages = static_cast<int>((k + pair::BK - 1) / pair::BK);
     p.y = y;
     p.ldy = ldy;

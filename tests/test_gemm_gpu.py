@@ -60,6 +60,7 @@ def _layer(nv, xb, wb, seg_offsets, rows=None, act_static=None, flags=0):
     (257, 520, 320, [0, 256, 520]),
     (64, 1040, 2048, [0, 512, 768, 1024, 1040]),
     (130, 264, 5120, [0, 136, 264]),
+    (8300, 600, 256, [0, 264, 600]),  # 33 M tiles: tile groups of 16, 16 and a ragged 1
 ])
 def test_gemm_parity_random(nv, m, n, k, segs):
     import torch
