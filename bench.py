@@ -119,12 +119,6 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- helpers
 
-def dev_bf16_from_bits(bits):
-    import numpy as np
-    import torch
-    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
-
-
 def gen_device(shape, dist, seed, outlier_frac=0.0, outlier_mult=1.0, sigma=1.0):
     """Seeded synthetic bf16 tensor generated on the GPU (Philox), with the
     workloads' distributions: N(0, sigma) or Student-t nu=3, plus scaled
