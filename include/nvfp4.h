@@ -145,7 +145,15 @@ nvfp4_status nvfp4_pack_weight(const void *w, int64_t n, int64_t k, int64_t ldw,
  * seg_gscales   device float[nseg] weight global scale per segment.
  * y             device [m, n] output (bf16, or fp32 with NVFP4_FLAG_F32_OUT), row stride ldy.
  * flags         NVFP4_FLAG_* bits.
- * Needs no workspace. */
+ * Needs no workspace.
+ * Errors (host-checked, nothing enqueued): NVFP4_ERR_INVALID_ARG for m < 0,
+ * n <= 0, k <= 0, an unknown flag bit, a NULL operand (activation operands and
+ * y may be NULL only when m == 0), ldy < n, or a malformed segment table;
+ * NVFP4_ERR_UNSUPPORTED_SHAPE for k % 64 != 0, n % 8 != 0, an interior segment
+ * offset not a multiple of 8, nseg > NVFP4_MAX_SEGMENTS, or sizes beyond the
+ * 32-bit tile indexing; NVFP4_ERR_MISALIGNED for an operand or y not 16-byte
+ * aligned or a y row stride not a multiple of 16 bytes.  A wait that runs out
+ * on the GPU shows up later as NVFP4_ERR_TIMEOUT from nvfp4_get_device_error. */
 nvfp4_status nvfp4_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m,
                         const uint8_t *qw, const uint8_t *sfw, int64_t n, int64_t k,
                         const int64_t *seg_offsets, const float *seg_gscales, int nseg,
@@ -162,7 +170,12 @@ nvfp4_status nvfp4_linear(const void *x, int64_t m, int64_t k, int64_t ldx, cons
 /* The whole layer for modules fused along N (e.g. q/k/v/gate projections
  * concatenated into one GEMM), each keeping its own weight global scale:
  * column j of segment i is scaled by s_x * seg_gscales[i] (paper §6).
- * seg_offsets host int64[nseg+1]; seg_gscales device float[nseg]. */
+ * seg_offsets host int64[nseg+1]; seg_gscales device float[nseg].
+ * Errors: those of nvfp4_gemm for the GEMM's arguments and of
+ * nvfp4_quantize_act for x, plus NVFP4_ERR_WORKSPACE for a NULL, unaligned or
+ * too small workspace.  A non-finite activation amax or act_gscale is reported
+ * by nvfp4_get_device_error as NVFP4_ERR_NONFINITE (the codes are then those of
+ * scale 0). */
 nvfp4_status nvfp4_linear_fused(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,
                                 const uint8_t *qw, const uint8_t *sfw, int64_t n,
                                 const int64_t *seg_offsets, const float *seg_gscales, int nseg,
