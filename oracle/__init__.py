@@ -63,6 +63,8 @@ def _load():
         lib.or_e2m1_encode_patterns.argtypes = [ctypes.c_uint64, ctypes.c_uint64, vp]
         lib.or_e2m1_encode_patterns.restype = None
         lib.or_e4m3_encode_patterns.argtypes, lib.or_e4m3_encode_patterns.restype = [vp, i64, vp], None
+        lib.or_e4m3_encode_range.argtypes = [ctypes.c_uint64, ctypes.c_uint64, vp]
+        lib.or_e4m3_encode_range.restype = None
         _lib = lib
     return _lib
 
@@ -94,6 +96,13 @@ def e2m1_encode_patterns(start: int, count: int) -> np.ndarray:
     """E2M1 codes of the fp32 bit patterns start .. start+count-1 (one byte each)."""
     out = np.empty(count, dtype=np.uint8)
     _load().or_e2m1_encode_patterns(start, count, _ptr(out))
+    return out
+
+
+def e4m3_encode_range(start: int, count: int) -> np.ndarray:
+    """E4M3 codes of the fp32 bit patterns start .. start+count-1 (one byte each)."""
+    out = np.empty(count, dtype=np.uint8)
+    _load().or_e4m3_encode_range(start, count, _ptr(out))
     return out
 
 

@@ -53,6 +53,9 @@
  *      largest scale as the shared one every ratio is <= 1, so no folded scale
  *      can pass 448 and the re-rounding error stays within E4M3's half ulp
  *      (2^-4 relative in the normal range; the paper reports <= 6.2%).
+ *      A NaN block-scale byte (0x7F or 0xFF; only a corrupt checkpoint holds
+ *      one) stays as it is: NaN times the ratio is NaN under IEEE rules, and
+ *      E4M3's NaN code keeps its sign bit.
  *  R16 Checkpoint import: a linear-layout block-scale matrix [rows, K/16]
  *      (one E4M3 byte per block, rows contiguous) is the logical matrix that
  *      R10 scatters; the packed codes need no change (same nibble order, R9).
@@ -389,7 +392,10 @@ float or_harmonize(uint8_t *sf, int64_t rows, int64_t k, const int64_t *seg_offs
         float ratio = seg_scale[i] / shared;                 /* fp32, <= 1 */
         for (int64_t r = seg_offsets[i]; r < seg_offsets[i + 1]; ++r)
             for (int64_t c = 0; c < nblk; ++c) {
-                float folded = (float)or_e4m3_value(sf[r * nblk + c]) * ratio;   /* fp32 product */
+                uint8_t b = sf[r * nblk + c];
+                if ((b & 0x7Fu) == 0x7Fu)     /* NaN code: NaN times the ratio is NaN, the byte stays */
+                    continue;
+                float folded = (float)or_e4m3_value(b) * ratio;   /* fp32 product */
                 sf[r * nblk + c] = (uint8_t)or_e4m3_encode(folded);
             }
     }
@@ -420,6 +426,49 @@ void or_e4m3_encode_patterns(const uint32_t *pats, int64_t count, uint8_t *out)
         float v;
         memcpy(&v, &pats[i], sizeof v);
         out[i] = (uint8_t)or_e4m3_encode(v);
+    }
+}
+
+/* out[i] = E4M3 code (R5) of the fp32 whose bit pattern is start + i, for
+ * whole ranges of patterns.  The rule is or_e4m3_encode's -- the nearest of
+ * the 127 finite non-negative E4M3 values to |v|, a tie to the even code,
+ * saturation at 448, the sign bit of v -- with the nearest value found by
+ * bisection over a table of those values instead of a scan. */
+void or_e4m3_encode_range(uint64_t start, uint64_t count, uint8_t *out)
+{
+    double tab[127];
+    for (uint32_t c = 0; c < 127; ++c)
+        tab[c] = or_e4m3_value(c);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < (int64_t)count; ++i) {
+        uint32_t u = (uint32_t)(start + (uint64_t)i);
+        float v;
+        memcpy(&v, &u, sizeof v);
+        uint32_t sign = signbit(v) ? 0x80u : 0u;
+        double a = fabs((double)v);
+        uint32_t code;
+        if (!(a <= tab[126])) {
+            code = 126;                       /* beyond 448 (or NaN): saturate */
+        } else {
+            uint32_t lo = 0, hi = 126;        /* invariant: tab[lo] <= a <= tab[hi] */
+            if (a == tab[0])
+                hi = 0;
+            while (hi - lo > 1) {
+                uint32_t mid = (lo + hi) / 2;
+                if (tab[mid] <= a)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            double dl = a - tab[lo], dh = tab[hi] - a;
+            if (dl < dh)
+                code = lo;
+            else if (dh < dl)
+                code = hi;
+            else
+                code = (lo & 1u) == 0 ? lo : hi;
+        }
+        out[i] = (uint8_t)(sign | code);
     }
 }
 

@@ -98,6 +98,40 @@ def test_e4m3_encode_saturates(oracle_mod):
         assert oracle_mod.e4m3_encode(v) == 0x7E
 
 
+def test_e4m3_range_encoder_matches_the_scan_and_torch(oracle_mod):
+    """The bulk E4M3 encoder over ranges of fp32 patterns (bisection over the
+    table of E4M3 values) gives the scan's codes on a stride through every
+    pattern of both signs, NaNs excluded, and torch's float8_e4m3fn cast
+    wherever that cast does not overflow (|v| <= 448); every tie and near-tie
+    of both signs is included."""
+    start, count, step = 0, 1 << 32, 65521
+    pats = np.arange(start, count, step, dtype=np.uint64).astype(np.uint32)
+    grid = np.array([oracle_mod.e4m3_value(c) for c in range(127)])
+    mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)
+    near = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e9))])
+    near = np.concatenate([near, -near]).view(np.uint32)
+    got = np.concatenate([oracle_mod.e4m3_encode_range(int(p), 1) for p in near] +
+                         [oracle_mod.e4m3_encode_range(0, 1 << 16)])
+    vals = np.concatenate([near, np.arange(0, 1 << 16, dtype=np.uint32)])
+    assert np.array_equal(got, oracle_mod.e4m3_encode_patterns(vals))
+    f = pats.view(np.float32)
+    pats = pats[~np.isnan(f)]
+    got = np.empty(pats.size, np.uint8)
+    for i, p in enumerate(pats):
+        got[i] = oracle_mod.e4m3_encode_range(int(p), 1)[0]
+    assert np.array_equal(got, oracle_mod.e4m3_encode_patterns(pats))
+    f = pats.view(np.float32)
+    ok = np.abs(f) <= 448.0
+    ref = torch.from_numpy(f[ok].copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got[ok], ref)
+    nf = near.view(np.float32)
+    inside = np.abs(nf) <= 448.0
+    assert inside.sum() > 700
+    ref = torch.from_numpy(nf[inside].copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got_near = np.concatenate([oracle_mod.e4m3_encode_range(int(p), 1) for p in near[inside]])
+    assert np.array_equal(got_near, ref)
+
+
 def test_e4m3_relative_rounding_error_closed_form(oracle_mod):
     """RNE to 3 mantissa bits: relative error <= 2^-4 in the normal range
     (the pages quote <= 6.2% for re-rounded block scales)."""

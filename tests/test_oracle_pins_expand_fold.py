@@ -192,6 +192,32 @@ def test_harmonize_rejects_non_finite_or_negative_scales(oracle_mod):
     assert shared == 0.0 and np.array_equal(new, sf)
 
 
+def test_harmonize_keeps_nan_scale_bytes(oracle_mod):
+    """A NaN block-scale byte (E4M3 0x7F, or 0xFF with the sign bit set), which
+    only a corrupt checkpoint could hold, stays as it is: NaN times any module
+    ratio is NaN under IEEE rules (checked here with NumPy's float32 product),
+    and E4M3's one NaN code per sign encodes it.  Every other byte folds exactly
+    as it does without the NaN bytes present."""
+    w, off = _fused_weight(13, [32, 48], 128, [0.02, 0.02 * 2.75])
+    s = oracle_mod.segment_scales(w, off)
+    q, sf = oracle_mod.quantize(w, oracle_mod.row_scales_from_segments(off, s))
+    planted = [(3, 5, 0x7F), (off[1] + 2, 0, 0xFF), (off[1] + 40, 7, 0x7F)]
+    sf_nan = sf.copy()
+    for r, c, b in planted:
+        sf_nan[r, c] = b
+    new, shared = oracle_mod.harmonize(sf, off, s)
+    new_nan, shared_nan = oracle_mod.harmonize(sf_nan, off, s)
+    assert shared_nan == shared
+    keep = np.ones(sf.shape, bool)
+    for r, c, b in planted:
+        seg = int(np.searchsorted(off, r, side="right")) - 1
+        ratio = np.float32(s[seg]) / np.float32(shared)
+        assert np.isnan(np.float32(oracle_mod.e4m3_value(b)) * ratio)
+        assert new_nan[r, c] == b
+        keep[r, c] = False
+    assert np.array_equal(new_nan[keep], new[keep])
+
+
 def test_harmonized_gemm_repairs_the_collapsed_mismatch(oracle_mod):
     """The paper's GEMM-level probe: serving a fused group with the largest
     module scale and unchanged block scales is off by the scale ratio
