@@ -33,11 +33,14 @@ constexpr int kThreads = 256;
 // ------------------------------------------------------------------ exact bf16 rounding
 
 // bf16 bits of the value p * s rounded once to nearest (ties to even), for p with
-// at most 24 significant bits and s any fp32.  The fp32 product hi is exact up to
-// its rounding error lo = fma(p, s, -hi); hi rounds to the same bf16 as p * s
-// unless hi sits exactly on a bf16 midpoint, where the sign of lo decides.  Tiny
-// products (below 2^-120, where lo may not be representable) go through fp64,
-// where the product is exact.
+// at most 6 significant bits (an E2M1 value times an E4M3 value) and s any fp32.
+// The exact product then has at most 30 significant bits, so the fp32 product hi
+// is exact up to its rounding error lo = fma(p, s, -hi) as long as the lowest of
+// those bits, 2^29 below the leading one, is not below fp32's smallest subnormal
+// 2^-149: i.e. for |hi| >= 2^-120.  hi rounds to the same bf16 as p * s unless hi
+// sits exactly on a bf16 midpoint, where the sign of lo decides.  Smaller
+// products go through fp64, where the product is exact.  (A p with more bits
+// would need a higher threshold: 2^-102 for 24 bits.)
 __device__ __forceinline__ uint32_t bf16_bits_of_product(float p, float s)
 {
     const float hi = __fmul_rn(p, s);
@@ -317,8 +320,10 @@ __global__ void __launch_bounds__(kThreads) harmonize_kernel(HarmonizeParams p)
         return;                                // leave the scales as they are
     if (state == 0) {
         for (int idx = threadIdx.x; idx < p.nseg * 256; idx += blockDim.x) {
-            const float folded = __fmul_rn(e4m3_to_f32(static_cast<uint32_t>(idx & 255)), s_ratio[idx >> 8]);
-            s_fold[idx >> 8][idx & 255] = static_cast<uint8_t>(f32_to_e4m3(folded));
+            const uint32_t b = static_cast<uint32_t>(idx & 255);
+            const float folded = __fmul_rn(e4m3_to_f32(b), s_ratio[idx >> 8]);
+            // A NaN byte (0x7F, 0xFF) stays as it is (NaN times the ratio is NaN).
+            s_fold[idx >> 8][b] = (b & 0x7Fu) == 0x7Fu ? static_cast<uint8_t>(b) : static_cast<uint8_t>(f32_to_e4m3(folded));
         }
         __syncthreads();
     }
@@ -333,6 +338,7 @@ __global__ void __launch_bounds__(kThreads) harmonize_kernel(HarmonizeParams p)
             const int w = static_cast<int>(u & 31);
             uint32_t words[4] = {v.x, v.y, v.z, v.w};
             int seg = 0;
+            uint32_t nan_bytes = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int64_t row = rb * 128 + j * 32 + w;
@@ -341,12 +347,18 @@ __global__ void __launch_bounds__(kThreads) harmonize_kernel(HarmonizeParams p)
                         ++seg;
                     const uint8_t *f = s_fold[seg];
                     const uint32_t x = words[j];
+                    // A byte of x is a NaN code iff its low 7 bits are all set:
+                    // t has a zero byte exactly there (zero-byte test on t).
+                    const uint32_t t = (x & 0x7F7F7F7Fu) ^ 0x7F7F7F7Fu;
+                    nan_bytes |= (t - 0x01010101u) & ~t & 0x80808080u;
                     words[j] = static_cast<uint32_t>(f[x & 0xFFu]) | (static_cast<uint32_t>(f[(x >> 8) & 0xFFu]) << 8) |
                                (static_cast<uint32_t>(f[(x >> 16) & 0xFFu]) << 16) |
                                (static_cast<uint32_t>(f[x >> 24]) << 24);
                 }
             }
             v = make_uint4(words[0], words[1], words[2], words[3]);
+            if (nan_bytes != 0)
+                raise_device_error(4u /* NVFP4_ERR_NONFINITE */);
         }
         reinterpret_cast<uint4 *>(p.sf_out)[u] = v;
     }

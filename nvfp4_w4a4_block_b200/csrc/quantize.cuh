@@ -59,7 +59,9 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float v)
     return h & 0xFFu;
 }
 
-// Exact decode of an E4M3 byte (sign ignored: block scales are non-negative).
+// Exact decode of an E4M3 byte, sign included (the quantizers' block scales are
+// non-negative; the expansion and harmonization of imported scales rely on a
+// sign-bit byte decoding to a negative value).  0x7F and 0xFF decode to NaN.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code)
 {
     uint32_t h2;

@@ -210,6 +210,25 @@ def test_harmonize_bad_scale_reports_and_leaves_scales(nv):
     assert np.array_equal(pw.sf.cpu().numpy(), phys)        # untouched
 
 
+def test_harmonize_nan_scale_bytes_stay_and_are_reported(nv):
+    """NaN block-scale bytes (0x7F, 0xFF) in the rows of a fused weight stay as
+    they are, as in the oracle; every other byte folds as usual, and the call
+    records NVFP4_ERR_NONFINITE (the weight cannot be served as it is)."""
+    import torch
+    _, off, s_w, q, sf = _fused_packed(61, [136, 120], 320, [1.0, 2.75])
+    sf = sf.copy()
+    for r, c, b in [(0, 0, 0x7F), (135, 19, 0xFF), (136, 4, 0x7F), (255, 11, 0xFF)]:
+        sf[r, c] = b
+    pw = nv.PackedWeight(_u8(q), _u8(oracle.sf_to_physical(sf, 320)), _f32(s_w), 256, 320, off)
+    hw = nv.harmonize_scales(pw)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.ERR_NONFINITE
+    assert nv.get_device_error() == nv.OK
+    new, shared = oracle.harmonize(sf, off, s_w)
+    assert np.array_equal(hw.sf.cpu().numpy(), oracle.sf_to_physical(new, 320))
+    assert hw.gscale.cpu().numpy()[0] == shared
+
+
 def test_harmonized_gemm_on_the_fused_qkv_gate_workload(nv):
     """The paper's GEMM-level probe at the fused q/k/v/gate shape (N = 10336,
     module scales spread ~1-8x), on 64 sampled activation rows: a single-scale

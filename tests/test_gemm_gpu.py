@@ -33,22 +33,27 @@ def _bf16_to_f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def _layer(nv, xb, wb, seg_offsets, rows=None, act_static=None, flags=0):
-    """Run the whole layer on the GPU; return (y_gpu [rows], oracle dict)."""
+def _layer(nv, xb, wb, seg_offsets, act_static=None, flags=0):
+    """Run the whole layer on the GPU; return (y_gpu, oracle dict, packed weight).
+    Both operands' codes, scale bytes and global scales are first asserted equal
+    to the oracle's, so any output error is the GEMM's."""
     import torch
     x = to_cuda_bf16(xb)
     pw = nv.pack_weight(to_cuda_bf16(wb), seg_offsets)
     g = None if act_static is None else torch.tensor([act_static], dtype=torch.float32, device="cuda")
     y = nv.linear_fused(x, pw, act_gscale=g, flags=flags)
+    qx, sfx, sx = nv.quantize_act(x, gscale=g)
     torch.cuda.synchronize()
     assert nv.get_device_error() == nv.OK
-    ref = oracle.linear_reference(xb, wb, seg_offsets, rows=rows, act_scale=act_static)
+    ref = oracle.linear_reference(xb, wb, seg_offsets, act_scale=act_static)
+    k = xb.shape[1]
     assert pw.gscale.cpu().numpy().tobytes() == ref["s_w"].tobytes()
-    if rows is None:
-        yg = y
-    else:
-        yg = y[torch.as_tensor(np.asarray(rows), device="cuda")]
-    return yg, ref, pw
+    assert np.array_equal(pw.q.cpu().numpy(), ref["qw"]), "weight codes differ"
+    assert np.array_equal(pw.sf.cpu().numpy(), oracle.sf_to_physical(ref["sfw"], k)), "weight scales differ"
+    assert np.float32(sx.item()).tobytes() == np.float32(ref["s_x"]).tobytes()
+    assert np.array_equal(qx.cpu().numpy(), ref["qx"]), "activation codes differ"
+    assert np.array_equal(sfx.cpu().numpy(), oracle.sf_to_physical(ref["sfx"], k)), "activation scales differ"
+    return y, ref, pw
 
 
 @pytest.mark.parametrize("m,n,k,segs", [
@@ -236,28 +241,68 @@ def _rows_sample(m, seed, n_rand):
                                      np.arange(max(0, m - 32), m)]))
 
 
+def _workload_layer(nv, wl, xb, rows=None):
+    """The whole layer on one workload, checked the way the tolerance reading
+    asks for it:
+      * codes and scale bytes of both operands equal the oracle's (weights in
+        full; activations in full, or on the sampled rows when `rows` is given,
+        the global scale always from the whole tensor);
+      * the fp32 output is within 1e-3 of max(|R|, row RMS) of the fp64 oracle;
+      * the bf16 output is within that plus its own rounding, and equals the
+        round-to-nearest-even bf16 of the same kernel's fp32 output bit for bit.
+    """
+    import torch
+    wb = wl.w()
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), wl.seg_offsets)
+    qx, sfx, sx = nv.quantize_act(x)
+    y32 = nv.linear_fused(x, pw, flags=nv.FLAG_F32_OUT)
+    ybf = nv.linear_fused(x, pw)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    ref = oracle.linear_reference(xb, wb, wl.seg_offsets, rows=rows)
+    # operands: bit-exact
+    assert pw.gscale.cpu().numpy().tobytes() == ref["s_w"].tobytes()
+    assert np.array_equal(pw.q.cpu().numpy(), ref["qw"]), "weight codes differ"
+    assert np.array_equal(pw.sf.cpu().numpy(), oracle.sf_to_physical(ref["sfw"], wl.k)), "weight scales differ"
+    assert np.float32(sx.item()).tobytes() == np.float32(ref["s_x"]).tobytes()
+    if rows is None:
+        assert np.array_equal(qx.cpu().numpy(), ref["qx"]), "activation codes differ"
+        assert np.array_equal(sfx.cpu().numpy(), oracle.sf_to_physical(ref["sfx"], wl.k)), "activation scales differ"
+        y32h, ybfh = y32.cpu().numpy(), ybf.view(torch.int16).cpu().numpy().view(np.uint16)
+    else:
+        sel = torch.as_tensor(np.asarray(rows), device="cuda")
+        assert np.array_equal(qx[sel].cpu().numpy(), ref["qx"]), "activation codes differ"
+        sf_h = sfx.cpu().numpy()
+        offs = np.array([[oracle.sf_offset(int(r), c, wl.k) for c in range(wl.k // 16)] for r in rows])
+        assert np.array_equal(sf_h[offs], ref["sfx"]), "activation scales differ"
+        y32h, ybfh = y32[sel].cpu().numpy(), ybf[sel].view(torch.int16).cpu().numpy().view(np.uint16)
+    # GEMM: fp32 within 1e-3, bf16 within 1e-3 + its rounding and equal to RNE(fp32)
+    assert_gemm_close(y32h, ref["y"], bf16=False)
+    assert_gemm_close(W.bf16_bits_to_f32(ybfh), ref["y"], bf16=True)
+    assert np.array_equal(ybfh, bf16_rne_from_f32(y32h))
+
+
 def test_tiny_workload_full(nv):
-    wl = W.TINY
-    y, ref, _ = _layer(nv, wl.x(), wl.w(), wl.seg_offsets)
-    assert_gemm_close(_bf16_to_f64(y), ref["y"], bf16=True)
+    _workload_layer(nv, W.TINY, W.TINY.x())
 
 
 @pytest.mark.parametrize("m", W.DECODE_M)
 def test_decode_workload_full(nv, m):
-    wl = W.DECODE
-    y, ref, _ = _layer(nv, wl.x(m), wl.w(), wl.seg_offsets)
-    assert_gemm_close(_bf16_to_f64(y), ref["y"], bf16=True)
+    _workload_layer(nv, W.DECODE, W.DECODE.x(m))
 
 
-@pytest.mark.parametrize("wl", [W.PREFILL, W.FUSED_QKVG], ids=lambda w: w.name)
-def test_prefill_workloads_sampled_rows(nv, wl):
-    rows = _rows_sample(wl.m, wl.cfg_id, 64)
-    y, ref, _ = _layer(nv, wl.x(), wl.w(), wl.seg_offsets, rows=rows)
-    assert_gemm_close(_bf16_to_f64(y), ref["y"], bf16=True)
+def test_fused_qkvg_workload_full(nv):
+    """4096 x 5120 -> 6144 + 2048 + 2048 + 96, four modules with their own
+    weight global scales: every output element against the oracle."""
+    _workload_layer(nv, W.FUSED_QKVG, W.FUSED_QKVG.x())
+
+
+def test_prefill_workload_sampled_rows(nv):
+    wl = W.PREFILL
+    _workload_layer(nv, wl, wl.x(), rows=_rows_sample(wl.m, wl.cfg_id, 64))
 
 
 def test_long_prefill_workload_sampled_rows(nv):
     wl = W.LONG_DOWN
-    rows = _rows_sample(wl.m, wl.cfg_id, 32)[::2]
-    y, ref, _ = _layer(nv, wl.x(), wl.w(), wl.seg_offsets, rows=rows)
-    assert_gemm_close(_bf16_to_f64(y), ref["y"], bf16=True)
+    _workload_layer(nv, wl, wl.x(), rows=_rows_sample(wl.m, wl.cfg_id, 32)[::2])

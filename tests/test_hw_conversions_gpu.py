@@ -9,13 +9,16 @@ converts every fp32 bit pattern of a range and the codes are compared byte for
 byte with the oracle's encoders:
 
   * E2M1: every finite pattern and both infinities (4.28e9 inputs);
-  * E4M3: every pattern in [0, 464] whose low 8 mantissa bits are zero, plus
-    each midpoint between neighbouring E4M3 values and its two fp32
-    neighbours (all tie and near-tie inputs).
+  * E4M3: every finite pattern of both signs and both infinities (the block
+    scales are non-negative; harmonization also folds sign-bit scale bytes of
+    imported checkpoints, whose products are negative), plus each midpoint
+    between neighbouring E4M3 values and its two fp32 neighbours listed on
+    their own.
 
 NaN inputs are not compared: no step of the layer feeds one to a conversion
 except a non-finite tensor, whose codes are unspecified (its amax is reported
-as non-finite).
+as non-finite), and harmonization keeps NaN scale bytes without converting
+them.
 """
 import ctypes
 import os
@@ -63,6 +66,24 @@ __global__ void e2m1_range_probe(unsigned long long start, unsigned long long gr
     }
 }
 
+// out[i] = E4M3 code of the fp32 with bits start + i; each thread converts
+// 4 consecutive patterns (two conversions of a pair each).
+__global__ void e4m3_range_probe(unsigned long long start, unsigned long long groups, unsigned int *out)
+{
+    const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
+    for (unsigned long long g = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x; g < groups; g += stride) {
+        const unsigned int u = (unsigned int)(start + 4ull * g);
+        unsigned int w = 0;
+        for (int j = 0; j < 2; ++j) {
+            unsigned short h;
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+                : "=h"(h) : "f"(__uint_as_float(u + 2 * j + 1)), "f"(__uint_as_float(u + 2 * j)));
+            w |= (unsigned int)h << (16 * j);
+        }
+        out[g] = w;
+    }
+}
+
 __global__ void e4m3_list_probe(const unsigned int *pats, long long count, unsigned char *out)
 {
     const long long stride = (long long)gridDim.x * blockDim.x;
@@ -77,6 +98,13 @@ extern "C" int probe_e2m1_range(unsigned long long start, unsigned long long cou
 {
     if (count % 8 != 0) return -1;
     e2m1_range_probe<<<1184, 256>>>(start, count / 8, (uint2 *)out);
+    return (int)cudaDeviceSynchronize();
+}
+
+extern "C" int probe_e4m3_range(unsigned long long start, unsigned long long count, void *out)
+{
+    if (count % 4 != 0) return -1;
+    e4m3_range_probe<<<1184, 256>>>(start, count / 4, (unsigned int *)out);
     return (int)cudaDeviceSynchronize();
 }
 
@@ -104,6 +132,7 @@ def probe(tmp_path_factory):
     vp, i64, u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64
     L.probe_e2m1_range.argtypes, L.probe_e2m1_range.restype = [u64, u64, vp], ctypes.c_int
     L.probe_e4m3_list.argtypes, L.probe_e4m3_list.restype = [vp, i64, vp], ctypes.c_int
+    L.probe_e4m3_range.argtypes, L.probe_e4m3_range.restype = [u64, u64, vp], ctypes.c_int
     return L
 
 
@@ -135,6 +164,22 @@ def test_e2m1_conversion_matches_oracle_on_every_finite_pattern(probe):
             got = out[:count].cpu().numpy()
             want = oracle.e2m1_encode_patterns(first, count)
             _first_mismatch(lambda i: first + i, got, want, "E2M1 code")
+
+
+def test_e4m3_conversion_matches_oracle_on_every_finite_pattern(probe):
+    import torch
+    chunk = 1 << 27
+    last = 0x7F800000                                   # +inf; the patterns above it are NaN
+    out = torch.empty(chunk, dtype=torch.uint8, device="cuda")
+    for sign in (0, 0x80000000):
+        for start in range(0, last + 1, chunk):
+            count = min(chunk, last + 1 - start)
+            first = sign + start
+            run = (count + 3) // 4 * 4                  # the probe converts runs of 4 patterns
+            assert probe.probe_e4m3_range(first, run, out.data_ptr()) == 0
+            got = out[:count].cpu().numpy()
+            want = oracle.e4m3_encode_range(first, count)
+            _first_mismatch(lambda i: first + i, got, want, "E4M3 code")
 
 
 def test_e4m3_conversion_matches_oracle_including_every_tie(probe):

@@ -253,9 +253,16 @@ def test_quantize_nonfinite_in_the_one_launch_path(nv, m, k):
     assert nv.get_device_error() == nv.OK
 
 
-@pytest.mark.parametrize("wl", [W.TINY, W.DECODE, W.PREFILL, W.FUSED_QKVG], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [W.TINY, W.PREFILL, W.FUSED_QKVG], ids=lambda w: w.name)
 def test_quantize_workload_activations(nv, wl):
     _compare(nv, wl.x())
+
+
+@pytest.mark.parametrize("m", W.DECODE_M)
+def test_quantize_decode_activations_every_token_count(nv, m):
+    """The decode activations at M = 1, 8 and 32 (the first rows of one draw):
+    each token count has its own dynamic global scale, so each is compared."""
+    _compare(nv, W.DECODE.x(m))
 
 
 def test_quantize_long_prefill_activations_sampled_rows(nv):
@@ -279,8 +286,10 @@ def test_quantize_long_prefill_activations_sampled_rows(nv):
     assert np.array_equal(sf_h[offs], sfo)
 
 
-@pytest.mark.parametrize("wl", [W.DECODE, W.FUSED_QKVG], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [W.TINY, W.DECODE, W.PREFILL, W.FUSED_QKVG, W.LONG_DOWN], ids=lambda w: w.name)
 def test_pack_weight_per_segment_scales(nv, wl):
+    """Every workload's packed weight, in full: per-segment global scales, codes
+    and scale bytes (pads included) equal to the oracle's."""
     import torch
     wb = wl.w()
     pw = nv.pack_weight(to_cuda_bf16(wb), wl.seg_offsets)
