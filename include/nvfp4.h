@@ -96,6 +96,10 @@ typedef enum {
                                                 writes no valid output and records NVFP4_ERR_TIMEOUT in
                                                 the device error word (pair it with a short
                                                 nvfp4_set_wait_timeout_ns).  No paper counterpart. */
+#define NVFP4_FLAG_TEST_STALL_LATE 0x200u    /* testing only, as NVFP4_FLAG_TEST_STALL but the stage
+                                                withheld is the last K stage of each CTA pair's second
+                                                output tile (of each CTA's tile in the decode kernel),
+                                                after earlier tiles completed.  No paper counterpart. */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *nvfp4_status_string(nvfp4_status st);
@@ -198,10 +202,12 @@ nvfp4_status nvfp4_linear_fused(const void *x, int64_t m, int64_t k, int64_t ldx
  * device array of NVFP4_NOALLOC_SCRATCH_BYTES inside the library instead of a
  * caller workspace; a problem whose nvfp4_workspace_bytes(m, n, k) exceeds that
  * size is rejected with NVFP4_ERR_SCRATCH_LIMIT before anything is enqueued
- * (at K = 5120 that allows up to about 2900 tokens).
+ * (at K = 5120 that allows up to 2895 tokens; 847 at K = 17408).  Malformed
+ * arguments get the status nvfp4_linear_fused would give them.
  *
  * The first call on a device looks up the array's device address (a one-time
- * set-up with that device current); make that first call before any stream
+ * set-up with that device current, made again if the device's context was
+ * replaced, e.g. by cudaDeviceReset); make that first call before any stream
  * capture.  The call allocates nothing.  All calls share the one array and it
  * keeps the last call's contents; nothing in it needs to start at zero.  Calls
  * whose work overlaps on the GPU (different streams without ordering between
@@ -264,8 +270,11 @@ nvfp4_status nvfp4_import_weight_scales(const uint8_t *sf_linear, int64_t n, int
  * shared_gscale_out device float, receives s_shared.
  * A negative or non-finite module scale leaves the scales unchanged, writes
  * NaN to *shared_gscale_out and records NVFP4_ERR_NONFINITE in the device error
- * word.  An all-zero group is left unchanged (s_shared = 0).  Pad rows are
- * copied unchanged.  Needs no workspace. */
+ * word.  A NaN block-scale byte (0x7F or 0xFF, which only a corrupt checkpoint
+ * holds) is kept as it is (NaN times the ratio is NaN) while the other bytes
+ * fold as usual, and the call records NVFP4_ERR_NONFINITE.  An all-zero group
+ * is left unchanged (s_shared = 0).  Pad rows are copied unchanged.  Needs no
+ * workspace. */
 nvfp4_status nvfp4_harmonize_scales(const uint8_t *sf_in, uint8_t *sf_out, int64_t n, int64_t k,
                                     const int64_t *seg_offsets, const float *seg_gscales, int nseg,
                                     float *shared_gscale_out, nvfp4_stream_t stream);
@@ -285,6 +294,25 @@ void nvfp4_set_wait_timeout_ns(uint64_t ns);
  * device work, e.g. the launches recorded into a CUDA graph; the paper has no
  * counterpart. */
 uint64_t nvfp4_launch_count(void);
+
+/* Measurement helper, not a step of the layer: the dense block-scaled FP4
+ * tensor-core rate of this device, the denominator for the GEMM's "fraction of
+ * peak" (the paper's W4A4 GEMM runs on native 4-bit tensor cores, "Why Gated
+ * DeltaNet Survives 4-Bit Quantization", §2 "NVFP4"; it quotes no rate).
+ * Enqueues on `stream` one launch in which each of `pairs` CTA pairs (one CTA
+ * per SM; at most half the SM count) issues `iters` x 4 of the GEMM's own
+ * instruction, tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 with
+ * M = 256, N = 256, K = 64, into one accumulator from operands and scales
+ * resident in shared memory -- no global-memory traffic.  With
+ * with_scale_copies != 0 every four MMAs are preceded by the GEMM's three
+ * per-stage scale-factor copies into tensor memory.  *flops receives the
+ * launch's MMA flops (2 * 256 * 256 * 64 * 4 * iters * pairs); time the launch
+ * with CUDA events on `stream`.  Keep one launch under a few seconds: its final
+ * wait is bounded at 10 s and then records NVFP4_ERR_TIMEOUT.  Errors:
+ * NVFP4_ERR_INVALID_ARG (pairs < 1, iters < 1, flops NULL),
+ * NVFP4_ERR_UNSUPPORTED_SHAPE (more pairs than SMs / 2). */
+nvfp4_status nvfp4_mma_peak_probe(int pairs, int64_t iters, int with_scale_copies, double *flops,
+                                  nvfp4_stream_t stream);
 
 /* Library version string. */
 const char *nvfp4_version(void);

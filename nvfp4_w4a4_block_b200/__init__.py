@@ -42,12 +42,14 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 FLAG_F32_OUT = 0x1
 FLAG_COLLAPSED_MAX_SCALE = 0x2
 FLAG_TEST_STALL = 0x100
+FLAG_TEST_STALL_LATE = 0x200
 MAX_SEGMENTS = 8
 
 EXPORTED = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize_act",
             "nvfp4_pack_weight", "nvfp4_gemm", "nvfp4_linear", "nvfp4_linear_fused", "nvfp4_get_device_error",
             "nvfp4_set_wait_timeout_ns", "nvfp4_version", "nvfp4_linear_fused_noalloc", "nvfp4_dequantize",
-            "nvfp4_import_weight_scales", "nvfp4_harmonize_scales", "nvfp4_launch_count")
+            "nvfp4_import_weight_scales", "nvfp4_harmonize_scales", "nvfp4_launch_count",
+            "nvfp4_mma_peak_probe")
 
 
 class NVFP4Error(RuntimeError):
@@ -98,6 +100,8 @@ def lib() -> ctypes.CDLL:
                 L.nvfp4_import_weight_scales.restype = ci
                 L.nvfp4_harmonize_scales.argtypes = [vp, vp, i64, i64, vp, vp, ci, vp, vp]
                 L.nvfp4_harmonize_scales.restype = ci
+                L.nvfp4_mma_peak_probe.argtypes = [ci, i64, ci, ctypes.POINTER(ctypes.c_double), vp]
+                L.nvfp4_mma_peak_probe.restype = ci
                 _lib = L
     return _lib
 
@@ -331,4 +335,18 @@ def harmonize_scales(pw: PackedWeight, in_place: bool = False, stream=None) -> P
                                       _stream(stream))
     _check(st, "nvfp4_harmonize_scales")
     return PackedWeight(pw.q, sf, shared, pw.n, pw.k, [0, pw.n])
+
+
+def mma_peak_probe(iters: int, pairs: Optional[int] = None, with_scale_copies: bool = False, stream=None) -> float:
+    """Enqueue one launch of the dense FP4 tensor-core probe (measurement only,
+    see nvfp4_mma_peak_probe) and return its MMA flops; time it with CUDA events
+    on the same stream.  pairs defaults to half the SM count (every SM)."""
+    torch = _torch()
+    if pairs is None:
+        pairs = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count // 2
+    flops = ctypes.c_double(0.0)
+    st = lib().nvfp4_mma_peak_probe(int(pairs), int(iters), 1 if with_scale_copies else 0, ctypes.byref(flops),
+                                    _stream(stream))
+    _check(st, "nvfp4_mma_peak_probe")
+    return flops.value
 

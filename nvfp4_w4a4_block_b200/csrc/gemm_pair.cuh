@@ -64,8 +64,9 @@ constexpr int OFF_STG = OFF_SFB + STAGES * SFB_BYTES;   // bf16 output staging: 
 constexpr int STG_SUB = 128 * 64 * 2;
 constexpr int OFF_BAR = OFF_STG + 2 * STG_SUB;
 constexpr int NUM_BARS = 2 * STAGES + 3;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_ALLOC = OFF_MISC + 64 + 1024;
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // +0 TMEM base, +4 abort flag, +8 peer's abort flag, +16 alpha[8]
+constexpr int OFF_DRAIN = OFF_MISC + 64;            // copy records (struct Drain)
+constexpr int SMEM_ALLOC = OFF_DRAIN + 128 + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert(TMEM_SFB + KB * 8 <= TMEM_COLS, "tensor memory budget");
 
@@ -84,8 +85,41 @@ struct Params {
     int seg_end[8];
     unsigned flags;
     uint64_t timeout_ns;
-    int stall_stage;             // testing: K stage of each pair's first tile whose loads are withheld (-1: none)
+    int stall_tile;              // testing: a K stage of each pair's tile number stall_tile (0 = its first tile)
+    int stall_stage;             //   has its loads withheld: stage stall_stage (-1: none)
 };
+
+// What a CTA's producer put in flight, per ring slot: the newest stage (by
+// sequence number q = tile iteration * k_stages + ks; slot q % STAGES, barrier
+// phase (q / STAGES) & 1) it issued copies for, the bytes of those copies, and,
+// in the even CTA, whether that stage's barrier was armed with both CTAs'
+// bytes.  Only a slot's newest stage can have copies in flight: a slot is
+// reused only after the MMAs consumed its previous stage, i.e. after every byte
+// of it landed.  At exit the odd CTA copies its records into peer_* of the even
+// CTA, whose stage barriers count both CTAs' copies, so that after a timeout
+// the even CTA can wait for exactly the copies still in flight.
+struct Drain {
+    int seq[STAGES];
+    uint32_t bytes[STAGES];
+    uint32_t armed[STAGES];
+    int peer_seq[STAGES];
+    uint32_t peer_bytes[STAGES];
+};
+static_assert(sizeof(Drain) <= 128, "copy records fit their slot");
+
+// Records that this CTA issues `bytes` more for stage sequence number q.
+__device__ __forceinline__ void note_issue(Drain *d, int q, uint32_t bytes, bool armed)
+{
+    const int s = q % STAGES;
+    if (d->seq[s] != q) {
+        d->seq[s] = q;
+        d->bytes[s] = 0;
+        d->armed[s] = 0;
+    }
+    d->bytes[s] += bytes;
+    if (armed)
+        d->armed[s] = 1;
+}
 
 // Segment (module) of output column `col`.
 __device__ __forceinline__ int col_segment(const Params &p, int col)
@@ -140,6 +174,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint64_t *final_bar = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    volatile int *peer_abort = reinterpret_cast<volatile int *>(smem + OFF_MISC + 8);
+    Drain *drain = reinterpret_cast<Drain *>(smem + OFF_DRAIN);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -157,6 +193,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         mbar_init(acc_empty, 2 * EPI_WARPS);
         mbar_init(final_bar, 1);
         *abort_flag = 0;
+        *peer_abort = 0;
+        for (int s = 0; s < STAGES; ++s) {
+            drain->seq[s] = -1;
+            drain->bytes[s] = 0;
+            drain->armed[s] = 0;
+            drain->peer_seq[s] = -1;
+            drain->peer_bytes[s] = 0;
+        }
         fence_barrier_init();
         prefetch_tensormap(&tm_a);
         prefetch_tensormap(&tm_b);
@@ -196,8 +240,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tile_coords(p, pair_id, mb0, nb);
             const int row_b = nb * BN + static_cast<int>(rank) * 128;
             for (int ks = 0; ks < pre; ++ks) {
-                if (ks != p.stall_stage && elect_one()) {
+                if (!(p.stall_tile == 0 && ks == p.stall_stage) && elect_one()) {
                     const uint32_t bar = bar0 + ks * 8;
+                    note_issue(drain, ks, B_BYTES + SFB_BYTES, rank == 0);
                     if (rank == 0)
                         mbar_arrive_expect_tx(&full[ks], TX_BYTES);
                     tma_load_2d_pair_hint(smem + OFF_B + ks * B_BYTES, &tm_b, ks * (BK / 2), row_b, bar, keep);
@@ -207,7 +252,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
         }
         pdl_wait_prerequisites();                        // the activation codes and scales are written
-        for (int tile = pair_id; tile < num_tiles && ok; tile += npairs) {
+        int it = 0;                                      // this pair's tile iteration
+        for (int tile = pair_id; tile < num_tiles && ok; tile += npairs, ++it) {
             int mb, nb;
             tile_coords(p, tile, mb, nb);
             const int row_a = mb * BM + static_cast<int>(rank) * 128;
@@ -217,9 +263,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (!ok)
                     break;
                 const uint32_t bar = bar0 + stage * 8;
-                const bool withhold = tile == pair_id && ks == p.stall_stage;
-                const bool weights_issued = tile == pair_id && ks < pre;
+                const bool withhold = it == p.stall_tile && ks == p.stall_stage;
+                const bool weights_issued = it == 0 && ks < pre;
                 if (!withhold && elect_one()) {
+                    note_issue(drain, it * p.k_stages + ks, weights_issued ? A_BYTES + SFA_BYTES : STAGE_BYTES,
+                               rank == 0 && !weights_issued);
                     if (rank == 0 && !weights_issued)
                         mbar_arrive_expect_tx(&full[stage], TX_BYTES);
                     tma_load_2d_pair_hint(smem + OFF_A + stage * A_BYTES, &tm_a, ks * (BK / 2), row_a, bar, keep);
@@ -241,12 +289,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // into the slots this grid frees (it waits for this grid's completion
         // before it reads anything this grid writes).
         pdl_launch_dependents();
-        if (!ok) {
-            // Give copies already issued time to land before the CTA can exit.
-            const uint64_t t0 = global_timer_ns();
-            while (global_timer_ns() - t0 < 100000ull) {
-            }
-        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (even CTA)
         // The whole warp runs the loop; an elected lane issues the scale copies,
@@ -434,16 +476,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (*abort_flag) {
-        // A role gave up: copies it or another role issued may still be landing
-        // (their barriers are no longer waited on).  Give them time before the
-        // shared memory and tensor memory are released.
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 100000ull) {
+    // Every role of this CTA is done.  Each CTA tells the other whether it gave
+    // up, and the odd CTA hands its copy records to the even one.
+    if (threadIdx.x == 0) {
+        st_cluster_u32(map_to_rank(smem_u32(const_cast<int *>(peer_abort)), rank ^ 1u), *abort_flag ? 1u : 0u);
+        if (rank == 1) {
+            for (int s = 0; s < STAGES; ++s) {
+                st_cluster_u32(map_to_rank(smem_u32(&drain->peer_seq[s]), 0), static_cast<uint32_t>(drain->seq[s]));
+                st_cluster_u32(map_to_rank(smem_u32(&drain->peer_bytes[s]), 0), drain->bytes[s]);
+            }
         }
     }
     __syncwarp();
-    cluster_sync_all();                                 // the peer's MMAs and copies are finished
+    cluster_sync_all();                                 // the peer's MMAs are finished; the records are visible
+    if (*abort_flag || *peer_abort) {
+        // A role gave up, so some stage barriers were left unobserved and copies
+        // issued by either CTA may still be landing in its shared memory.  Both
+        // CTAs' copies complete on the even CTA's stage barriers: for each ring
+        // slot's newest stage the even CTA accounts for the bytes that were
+        // expected but never sent (or arms the stage with the bytes the odd CTA
+        // sent without it), then waits, bounded, until the phase completes --
+        // that is, until every copy of that stage has landed.  The odd CTA waits
+        // at the cluster barrier meanwhile.
+        if (rank == 0 && threadIdx.x == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                const int q0 = drain->seq[s], q1 = drain->peer_seq[s];
+                const int q = max(q0, q1);
+                if (q < 0)
+                    continue;
+                const uint32_t b = (q0 == q ? drain->bytes[s] : 0u) + (q1 == q ? drain->peer_bytes[s] : 0u);
+                if (q0 == q && drain->armed[s] != 0) {
+                    if (b < TX_BYTES)
+                        mbar_complete_tx(&full[s], TX_BYTES - b);
+                } else if (b != 0) {
+                    mbar_arrive_expect_tx(&full[s], b);
+                } else {
+                    continue;
+                }
+                volatile int no_abort = 0;
+                mbar_wait_bounded(&full[s], static_cast<uint32_t>((q / STAGES) & 1), &no_abort, DRAIN_TIMEOUT_NS);
+            }
+        }
+        __syncwarp();
+        cluster_sync_all();                             // no copy is in flight into either CTA
+    }
     if (threadIdx.x == 0 && *abort_flag)
         atomicCAS(&g_device_error, 0u, 6u /* NVFP4_ERR_TIMEOUT */);
     if (warp == 1) {

@@ -21,6 +21,7 @@
 #include "convert.cuh"
 #include "gemm_decode.cuh"
 #include "gemm_pair.cuh"
+#include "mma_peak.cuh"
 #include "quantize.cuh"
 
 // Device scratch of nvfp4_linear_fused_noalloc (see include/nvfp4.h).  In host
@@ -41,6 +42,7 @@ std::atomic<uint64_t> g_launches{0};       // kernel launches enqueued by this l
 
 struct DeviceInfo {
     bool ready = false;
+    unsigned long long ctx_id = 0;  // context the set-up below was made in
     nvfp4_status status = NVFP4_OK;
     int sms = 0;
     int tile_quant_ctas_per_sm = 1;
@@ -58,6 +60,37 @@ constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder bel
 // registers (quantize_cluster_kernel) up to this many elements.
 constexpr int64_t kClusterQuantElems = int64_t(kClusterCtas) * kClusterThreads * kClusterUnits * 8;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_get_id = nullptr;
+
+// Unique id of the calling thread's current CUDA context on device `dev`,
+// initialising the device's primary context first if no context is current.
+// Per-device state (kernel attributes, the scratch address) is keyed by it: a
+// cudaDeviceReset replaces the primary context, and everything set up in the
+// old one is gone, so a new id means the set-up is made again.  Called with
+// g_mu held.
+nvfp4_status current_context_id(int dev, unsigned long long *id)
+{
+    if (g_ctx_current == nullptr || g_ctx_get_id == nullptr) {
+        cudaDriverEntryPointQueryResult q1, q2;
+        void *f1 = nullptr, *f2 = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || f1 == nullptr ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess || f2 == nullptr)
+            return NVFP4_ERR_CUDA;
+        g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f1);
+        g_ctx_get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f2);
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS)
+        return NVFP4_ERR_CUDA;
+    if (ctx == nullptr) {
+        if (cudaSetDevice(dev) != cudaSuccess || g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+            return NVFP4_ERR_CUDA;
+    }
+    return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -88,8 +121,8 @@ cudaError_t launch(void (*kernel)(KArgs...), int grid, int block, size_t smem, c
     return e;
 }
 
-// One-time per-device set-up: capability check, SM count, kernel attributes,
-// driver entry point for tensor-map encoding.
+// One-time per-device (per-context) set-up: capability check, SM count, kernel
+// attributes, driver entry point for tensor-map encoding.
 nvfp4_status device_setup(int *sms)
 {
     int dev = 0;
@@ -97,7 +130,13 @@ nvfp4_status device_setup(int *sms)
         return NVFP4_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceInfo &d = g_dev[dev];
+    unsigned long long ctx_id = 0;
+    if (current_context_id(dev, &ctx_id) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
+    if (d.ready && d.ctx_id != ctx_id)
+        d.ready = false;                 // the context was replaced (cudaDeviceReset): set up again
     if (!d.ready) {
+        d.ctx_id = ctx_id;
         int major = 0, minor = 0, sm = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -117,7 +156,9 @@ nvfp4_status device_setup(int *sms)
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Cfg<32>::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode::Cfg<64>::SMEM_ALLOC) != cudaSuccess)
+                                 decode::Cfg<64>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(peak::mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 peak::SMEM_ALLOC) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         if (g_encode == nullptr) {
             cudaDriverEntryPointQueryResult q;
@@ -388,7 +429,17 @@ nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x
         p.seg_end[s] = static_cast<int>(seg_ends[s]);
     p.flags = flags;
     p.timeout_ns = g_timeout_ns.load();
-    p.stall_stage = (flags & NVFP4_FLAG_TEST_STALL) ? 1 : -1;
+    // Testing hooks: withhold the second K stage of each pair's first tile, or
+    // the last K stage of each pair's second tile.
+    p.stall_tile = -1;
+    p.stall_stage = -1;
+    if (flags & NVFP4_FLAG_TEST_STALL) {
+        p.stall_tile = 0;
+        p.stall_stage = 1;
+    } else if (flags & NVFP4_FLAG_TEST_STALL_LATE) {
+        p.stall_tile = 1;
+        p.stall_stage = p.k_stages - 1;
+    }
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
     return cuda_status(launch(pair::nvfp4_gemm_pair_kernel, static_cast<int>(2 * pairs), pair::THREADS,
@@ -426,7 +477,8 @@ nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s
         p.seg_end[s] = static_cast<int>(seg_ends[s]);
     p.flags = flags;
     p.timeout_ns = g_timeout_ns.load();
-    p.stall_stage = (flags & NVFP4_FLAG_TEST_STALL) ? 1 : -1;
+    // Testing hooks (one tile per CTA): withhold the second or the last K stage.
+    p.stall_stage = (flags & NVFP4_FLAG_TEST_STALL) ? 1 : (flags & NVFP4_FLAG_TEST_STALL_LATE) ? p.k_stages - 1 : -1;
     const int grid = static_cast<int>((n + decode::BW - 1) / decode::BW);
     return cuda_status(launch(decode::nvfp4_gemm_decode_kernel<T>, grid, decode::THREADS, decode::Cfg<T>::SMEM_ALLOC,
                               stream, pdl, tw, tx, p));
@@ -473,7 +525,8 @@ nvfp4_status check_gemm_args(const uint8_t *qx, const uint8_t *sfx, const float 
 {
     if (m < 0 || n <= 0 || k <= 0)
         return NVFP4_ERR_INVALID_ARG;
-    if (flags & ~(NVFP4_FLAG_F32_OUT | NVFP4_FLAG_COLLAPSED_MAX_SCALE | NVFP4_FLAG_TEST_STALL))
+    if (flags & ~(NVFP4_FLAG_F32_OUT | NVFP4_FLAG_COLLAPSED_MAX_SCALE | NVFP4_FLAG_TEST_STALL |
+                  NVFP4_FLAG_TEST_STALL_LATE))
         return NVFP4_ERR_INVALID_ARG;
     if (k % 64 != 0 || n % 8 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -654,25 +707,33 @@ nvfp4_status nvfp4_linear_fused_noalloc(const void *x, int64_t m, int64_t k, int
                                         const int64_t *seg_offsets, const float *seg_gscales, int nseg,
                                         void *y, int64_t ldy, unsigned flags, nvfp4_stream_t stream)
 {
-    if (m < 0 || k <= 0 || k % 16 != 0)
-        return m < 0 || k <= 0 ? NVFP4_ERR_INVALID_ARG : NVFP4_ERR_UNSUPPORTED_SHAPE;
+    // The shape is validated first, so a malformed call gets the same status as
+    // from nvfp4_linear_fused; only a well-formed problem too large for the
+    // scratch array gets NVFP4_ERR_SCRATCH_LIMIT.
+    nvfp4_status st = check_bf16_operand(x, m, k, ldx);
+    if (st != NVFP4_OK)
+        return st;
     if (workspace_layout(m, k).total > NVFP4_NOALLOC_SCRATCH_BYTES)
         return NVFP4_ERR_SCRATCH_LIMIT;
-    // One-time per-device look-up of the scratch array's device address, made
-    // with that device current.
-    static std::mutex mu;
+    // Per-device look-up of the scratch array's device address, made with that
+    // device current, once per context (again after a cudaDeviceReset).
     static void *scratch[64] = {};
+    static unsigned long long scratch_ctx[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return NVFP4_ERR_CUDA;
     void *ptr = nullptr;
     {
-        std::lock_guard<std::mutex> lock(mu);
-        if (scratch[dev] == nullptr) {
+        std::lock_guard<std::mutex> lock(g_mu);
+        unsigned long long ctx_id = 0;
+        if (current_context_id(dev, &ctx_id) != NVFP4_OK)
+            return NVFP4_ERR_CUDA;
+        if (scratch[dev] == nullptr || scratch_ctx[dev] != ctx_id) {
             void *p = nullptr;
             if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
                 return NVFP4_ERR_CUDA;
             scratch[dev] = p;
+            scratch_ctx[dev] = ctx_id;
         }
         ptr = scratch[dev];
     }
@@ -800,6 +861,24 @@ nvfp4_status nvfp4_harmonize_scales(const uint8_t *sf_in, uint8_t *sf_out, int64
     const int grid = static_cast<int>(blocks < cap ? blocks : cap);
     return cuda_status(launch(convert::harmonize_kernel, grid, convert::kThreads, 0,
                               reinterpret_cast<cudaStream_t>(stream), false, hp));
+}
+
+nvfp4_status nvfp4_mma_peak_probe(int pairs, int64_t iters, int with_scale_copies, double *flops,
+                                  nvfp4_stream_t stream)
+{
+    if (pairs < 1 || iters < 1 || iters > (int64_t(1) << 40) || flops == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    int sms = 0;
+    nvfp4_status st = device_setup(&sms);
+    if (st != NVFP4_OK)
+        return st;
+    if (pairs > sms / 2)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    st = cuda_status(launch(peak::mma_peak_kernel, 2 * pairs, peak::THREADS, peak::SMEM_ALLOC,
+                            reinterpret_cast<cudaStream_t>(stream), false, iters, with_scale_copies ? 1 : 0));
+    if (st == NVFP4_OK)
+        *flops = 2.0 * 256.0 * 256.0 * 64.0 * peak::KB * static_cast<double>(iters) * pairs;
+    return st;
 }
 
 nvfp4_status nvfp4_get_device_error(nvfp4_stream_t stream)

@@ -374,6 +374,20 @@ __device__ __forceinline__ void st_async_remote_u32(uint32_t cluster_addr, uint3
                  : "memory");
 }
 
+// Plain 32-bit store into the shared memory of a CTA of the cluster (address
+// from map_to_rank); ordered for the peer by the next cluster barrier.
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t value)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(value) : "memory");
+}
+
+// Counts `bytes` of the current phase's expected transaction bytes as arrived
+// without any copy (for bytes that were expected but will never be sent).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
 // Arrive on an mbarrier of another CTA of the cluster (address from map_to_rank).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 {

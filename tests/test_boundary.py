@@ -152,6 +152,26 @@ def test_harmonize_validation(L):
     assert f(FAKE, FAKE + 16, 64, 128, None, FAKE, 1, FAKE, None) == nv.ERR_INVALID_ARG    # partial overlap
 
 
+def test_noalloc_validation_and_exact_scratch_limit(L):
+    """The no-allocation entry checks the shape before its scratch limit (a
+    malformed call gets nvfp4_linear_fused's status), and at K = 5120 the
+    largest problem its 8 MiB scratch takes is 2895 tokens: 2896 is rejected on
+    the host with NVFP4_ERR_SCRATCH_LIMIT before any CUDA call."""
+    f = L.nvfp4_linear_fused_noalloc
+
+    def call(m, k, x=FAKE, ldx=None):
+        return f(x, m, k, k if ldx is None else ldx, None, FAKE, FAKE, 64, None, FAKE, 1, FAKE, 64, 0, None)
+
+    assert call(100000, 96) == nv.ERR_UNSUPPORTED_SHAPE          # K % 64 before the size limit
+    assert call(100000, 128, x=MIS) == nv.ERR_MISALIGNED
+    assert call(100000, 128, ldx=64) == nv.ERR_INVALID_ARG
+    assert call(-1, 128) == nv.ERR_INVALID_ARG
+    assert call(2896, 5120) == nv.ERR_SCRATCH_LIMIT
+    assert call(848, 17408) == nv.ERR_SCRATCH_LIMIT
+    assert nv.workspace_bytes(2895, 0, 5120) <= nv.NOALLOC_SCRATCH_BYTES < nv.workspace_bytes(2896, 0, 5120)
+    assert nv.workspace_bytes(847, 0, 17408) <= nv.NOALLOC_SCRATCH_BYTES < nv.workspace_bytes(848, 0, 17408)
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     mod = importlib.import_module("nvfp4_w4a4_block_b200")

@@ -48,3 +48,58 @@ def test_gemm_wait_timeout_is_reported_and_the_context_stays_usable(nv, m):
     assert nv.get_device_error() == nv.OK
     ref = oracle.linear_reference(xb, wb, off)
     assert_gemm_close(y.cpu().numpy(), ref["y"], bf16=False)
+
+
+def test_pair_gemm_late_stall_drains_and_the_context_stays_usable(nv):
+    """The CTA-pair kernel withholds the last K stage of each pair's second
+    output tile, after the first tile was stored: the MMA issuer's wait runs
+    out, the pair accounts for the copies of every ring slot and waits for
+    those in flight before it releases its memory, and the same context then
+    computes the right answer.  600 x 7680 gives 90 output tiles over the 74
+    pairs, so some pairs have a second tile."""
+    import torch
+    m, n, k = 600, 7680, 1344
+    xb, wb, off = W.random_case(77, m, n, k, seg_rows=[3840, 3840])
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    qx, sfx, sx = nv.quantize_act(x)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    nv.set_wait_timeout_ns(2_000_000)
+    try:
+        for _ in range(2):                              # twice: the abort path leaves nothing behind
+            nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT | nv.FLAG_TEST_STALL_LATE)
+            assert nv.get_device_error() == nv.ERR_TIMEOUT
+            assert nv.get_device_error() == nv.OK
+    finally:
+        nv.set_wait_timeout_ns(2_000_000_000)
+    y = nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    ref = oracle.linear_reference(xb, wb, off)
+    assert_gemm_close(y.cpu().numpy(), ref["y"], bf16=False)
+
+
+@pytest.mark.parametrize("m", [8, 40], ids=["decode_T8", "decode_T64"])
+def test_decode_gemm_late_stall_is_reported(nv, m):
+    """The decode kernel withholding its last K stage: reported as a timeout,
+    and the next call is correct."""
+    import torch
+    n, k = 392, 1344
+    xb, wb, off = W.random_case(78 + m, m, n, k, seg_rows=[128, 264])
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    qx, sfx, sx = nv.quantize_act(x)
+    torch.cuda.synchronize()
+    nv.set_wait_timeout_ns(2_000_000)
+    try:
+        nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT | nv.FLAG_TEST_STALL_LATE)
+        assert nv.get_device_error() == nv.ERR_TIMEOUT
+    finally:
+        nv.set_wait_timeout_ns(2_000_000_000)
+    y = nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    ref = oracle.linear_reference(xb, wb, off)
+    assert_gemm_close(y.cpu().numpy(), ref["y"], bf16=False)
+

@@ -7,12 +7,13 @@ nvfp4_linear_fused_noalloc keeps its scratch in a static device array of the
 library instead of a caller workspace.  This test calls it through the C ABI
 twice in a row (the second call reuses the scratch the first one left behind)
 and checks each result against the workspace entry point nvfp4_linear_fused on
-the same inputs.  It runs last so that a failure here leaves every other test
+the same inputs, and the fp32 result against the CPU oracle as well.  It runs last so that a failure here leaves every other test
 already run; it passes alone in a fresh process as well as after the others.
 """
 import numpy as np
 import pytest
 
+import oracle
 from nvfp4_w4a4_block_b200 import workloads as W
 
 from _helpers import assert_gemm_close, to_cuda_bf16
@@ -38,6 +39,7 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(nv):
         xb, wb, off = W.random_case(40 + seed, m, n, k, seg_rows=segs)
         x = to_cuda_bf16(xb)
         pw = nv.pack_weight(to_cuda_bf16(wb), off)
+        expect = oracle.linear_reference(xb, wb, off)["y"]
         for flags in (nv.FLAG_F32_OUT, 0):
             ref = nv.linear_fused(x, pw, flags=flags)
             got = nv.linear_fused_noalloc(x, pw, flags=flags)
@@ -47,18 +49,21 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(nv):
             g = got.float().cpu().numpy().astype(np.float64)
             assert_gemm_close(g, r, bf16=(flags == 0))
             assert torch.equal(got, ref)          # same kernels, same inputs: identical bits
+            assert_gemm_close(g, expect, bf16=(flags == 0))
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(nv):
     import torch
     k = 5120
-    m = nv.NOALLOC_SCRATCH_BYTES // (k // 2) + 1          # codes alone exceed the scratch
+    m = 2896                                              # one token beyond the limit at K = 5120
     pw = nv.pack_weight(to_cuda_bf16(W.random_case(50, 1, 64, k)[1]))
     x = torch.zeros((m, k), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(nv.NVFP4Error) as err:
         nv.linear_fused_noalloc(x, pw)
     assert err.value.status == nv.ERR_SCRATCH_LIMIT
-    # a fitting problem still works afterwards
-    y = nv.linear_fused_noalloc(x[:8], pw)
-    torch.cuda.synchronize()
-    assert y.shape == (8, 64) and not torch.isnan(y.float()).any()
+    # the largest problem that fits, and a small one, still work afterwards
+    for rows in (m - 1, 8):
+        y = nv.linear_fused_noalloc(x[:rows], pw)
+        torch.cuda.synchronize()
+        assert nv.get_device_error() == nv.OK
+        assert y.shape == (rows, 64) and not (y.float() != 0).any()      # zero activations give zeros
