@@ -388,10 +388,17 @@ __device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes)
     asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-// Arrive on an mbarrier of another CTA of the cluster (address from map_to_rank).
+// Arrive on an mbarrier of a CTA of the cluster (address from map_to_rank),
+// with the instruction's default semantics (release at CTA scope).  Measured
+// in the pair GEMM's accumulator hand-off: the explicit .release.cluster form
+// made each arrival take effect ~1.1 us later, because it first waits for the
+// arriving thread's earlier memory operations to become visible cluster-wide.
+// Callers that need a peer CTA to see data they wrote must order it otherwise
+// (the hand-off only signals that tensor-memory loads, already waited for with
+// tcgen05.wait::ld, are complete).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx_u32(uint32_t bar, uint32_t bytes)
