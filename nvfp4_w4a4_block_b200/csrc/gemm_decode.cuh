@@ -12,11 +12,13 @@
 //   * One CTA owns one 128-row weight tile over the whole K; two CTAs fit on an SM,
 //     so N/128 tiles (272 for N = 34816) are all resident at once and each SM keeps
 //     2 x (STAGES-1) weight stages in flight.
-//   * The kernel is launched with programmatic stream serialization: the producer
-//     streams the first STAGES weight stages before griddepcontrol.wait, i.e. while
-//     the activation quantizer that precedes it is still running, then loads the
-//     activation stages; once it has issued its last load it lets the next kernel
-//     in the stream be scheduled.
+//   * The kernel is launched with programmatic stream serialization: its set-up
+//     (barriers, tensor memory, descriptor prefetch) overlaps the end of the
+//     preceding kernel, and no global memory is touched before griddepcontrol.wait
+//     -- except behind this library's activation quantizer, where the producer
+//     streams the first STAGES weight stages before the wait, i.e. while the
+//     quantizer is still running.  Once it has issued its last load it lets the
+//     next kernel in the stream be scheduled.
 //
 // Roles: warp 0 producer (TMA + bulk copies), warp 1 MMA issuer (one elected lane),
 // warps 2..5 epilogue (tcgen05.ld of the 128 x T accumulator, x alpha(n), the tile
@@ -81,6 +83,9 @@ struct Params {
     unsigned flags;
     uint64_t timeout_ns;
     int stall_stage;             // testing: K stage whose loads are withheld (-1: none)
+    int early_weights;           // 1: the first weight stages are requested before griddepcontrol.wait
+                                 //    (the preceding kernel is this library's quantizer, which writes
+                                 //    no weights); 0: no global access before the wait
 };
 
 template <int T>
@@ -128,7 +133,9 @@ __global__ void __launch_bounds__(THREADS, 2)
         // The whole warp walks the schedule (operands stay warp-uniform); one
         // elected lane issues the copies.
         const int pre = min(C::STAGES, p.k_stages);
-        // Weight stages first: they do not depend on the preceding kernel.
+        if (!p.early_weights)
+            pdl_wait_prerequisites();            // the predecessor may write any input
+        // Weight stages first: behind the quantizer they do not depend on the preceding kernel.
         for (int ks = 0; ks < pre; ++ks) {
             const int nkb = min(KB, static_cast<int>(p.atoms_k) - ks * KB);
             const uint8_t *sfw_src = p.sfw + (static_cast<int64_t>(blockIdx.x) * p.atoms_k + ks * KB) * 512;

@@ -16,9 +16,10 @@
 //     for 128 x 256 x 256 MACs, a third less than a single-CTA 128 x 256 tile.
 //   * Five 38 KB stages per CTA.  Both CTAs' TMA loads complete on the even CTA's
 //     stage barrier; the even CTA's tcgen05.commit releases the stage in both.
-//     Launched behind the activation quantizer with programmatic stream
-//     serialization, the producers request the weight tiles and scales of their
-//     first five stages before griddepcontrol.wait.
+//     Launched with programmatic stream serialization, the set-up overlaps the
+//     preceding kernel; behind this library's activation quantizer the producers
+//     also request the weight tiles and scales of their first five stages before
+//     griddepcontrol.wait (otherwise nothing global is touched before it).
 //   * Eight epilogue warps per CTA drain the accumulator into registers (128
 //     columns each), hand the tensor memory back to the MMA issuer at once, and
 //     only then scale and convert -- the next tile's MMAs overlap the rest of the
@@ -87,6 +88,8 @@ struct Params {
     uint64_t timeout_ns;
     int stall_tile;              // testing: a K stage of each pair's tile number stall_tile (0 = its first tile)
     int stall_stage;             //   has its loads withheld: stage stall_stage (-1: none)
+    int early_weights;           // 1: the first weight stages are requested before griddepcontrol.wait
+                                 //    (behind this library's quantizer); 0: no global access before it
 };
 
 // What a CTA's producer put in flight, per ring slot: the newest stage (by
@@ -235,6 +238,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // stage (no arrival, no copies) makes the MMA issuer's bounded wait on it
         // run out.
         const int pre = pair_id < num_tiles ? min(STAGES, p.k_stages) : 0;
+        if (!p.early_weights)
+            pdl_wait_prerequisites();                    // the predecessor may write any input
         {
             int mb0, nb;
             tile_coords(p, pair_id, mb0, nb);

@@ -393,8 +393,8 @@ nvfp4_status make_out_map(CUtensorMap *map, void *y, uint64_t m, uint64_t n, uin
 
 nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
                          const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
-                         const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms, bool pdl,
-                         cudaStream_t stream)
+                         const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms,
+                         bool early_weights, cudaStream_t stream)
 {
     CUtensorMap ta, tb, tsa, tsb, ty;
     memset(&ty, 0, sizeof ty);
@@ -429,6 +429,7 @@ nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x
         p.seg_end[s] = static_cast<int>(seg_ends[s]);
     p.flags = flags;
     p.timeout_ns = g_timeout_ns.load();
+    p.early_weights = early_weights ? 1 : 0;
     // Testing hooks: withhold the second K stage of each pair's first tile, or
     // the last K stage of each pair's second tile.
     p.stall_tile = -1;
@@ -443,13 +444,13 @@ nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
     return cuda_status(launch(pair::nvfp4_gemm_pair_kernel, static_cast<int>(2 * pairs), pair::THREADS,
-                              pair::SMEM_ALLOC, stream, pdl, ta, tb, tsa, tsb, ty, p));
+                              pair::SMEM_ALLOC, stream, true, ta, tb, tsa, tsb, ty, p));
 }
 
 template <int T>
 nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
                            const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
-                           const float *seg_gscales, void *y, int64_t ldy, unsigned flags, bool pdl,
+                           const float *seg_gscales, void *y, int64_t ldy, unsigned flags, bool early_weights,
                            cudaStream_t stream)
 {
     CUtensorMap tw, tx;
@@ -479,16 +480,19 @@ nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s
     p.timeout_ns = g_timeout_ns.load();
     // Testing hooks (one tile per CTA): withhold the second or the last K stage.
     p.stall_stage = (flags & NVFP4_FLAG_TEST_STALL) ? 1 : (flags & NVFP4_FLAG_TEST_STALL_LATE) ? p.k_stages - 1 : -1;
+    p.early_weights = early_weights ? 1 : 0;
     const int grid = static_cast<int>((n + decode::BW - 1) / decode::BW);
     return cuda_status(launch(decode::nvfp4_gemm_decode_kernel<T>, grid, decode::THREADS, decode::Cfg<T>::SMEM_ALLOC,
-                              stream, pdl, tw, tx, p));
+                              stream, true, tw, tx, p));
 }
 
 // GEMM + epilogue.  Up to 64 tokens take the swapped decode kernel, more take
-// the persistent CTA-pair kernel (256 x 256 tiles).  `pdl` is set only when the preceding
+// the persistent CTA-pair kernel (256 x 256 tiles).  Both are launched with
+// programmatic stream serialization and touch no global memory before
+// griddepcontrol.wait, except that `early_weights` (set only when the preceding
 // kernel in the stream is this library's quantizer, whose early trigger comes
-// after all earlier work has completed (the decode kernel reads weights before
-// it waits on that quantizer).
+// after all earlier work has completed) lets them request their first weight
+// stages before it.
 nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
                          const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
                          const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms, bool pdl,
