@@ -16,9 +16,9 @@
  *   2. block-scaled FP4 GEMM with FP32 accumulation on the tcgen05 tensor cores;
  *   3. an epilogue that multiplies each output column by s_x * s_w[segment]
  *      and writes bf16.  A fused GEMM over several modules concatenated along N
- *      keeps one weight global scale per module (segment); the paper's §6
- *      "Per-module calibration vs. fused-GEMM scaling" shows what goes wrong
- *      when those are collapsed to one.
+ *      keeps one weight global scale per module (segment); "Why Gated DeltaNet
+ *      Survives 4-Bit Quantization", §6 "Per-module calibration vs. fused-GEMM
+ *      scaling", shows what goes wrong when those are collapsed to one.
  *
  * Conventions for every entry point
  *   - All pointers marked "device" are CUDA device (or managed) pointers; the
@@ -90,7 +90,8 @@ typedef enum {
 /* Flags for nvfp4_gemm / nvfp4_linear / nvfp4_linear_fused. */
 #define NVFP4_FLAG_F32_OUT 0x1u              /* write fp32 instead of bf16 (numerics checks) */
 #define NVFP4_FLAG_COLLAPSED_MAX_SCALE 0x2u  /* negative control: every column uses s_x * max(s_w),
-                                                the mismatch of the paper's §6; never for serving */
+                                                the mismatch of "Why Gated DeltaNet Survives
+                                                4-Bit Quantization", §6; never for serving */
 #define NVFP4_FLAG_TEST_STALL 0x100u         /* testing only: the GEMM's producer withholds its second
                                                 K stage, so a bounded pipeline wait runs out; the call
                                                 writes no valid output and records NVFP4_ERR_TIMEOUT in
@@ -173,7 +174,8 @@ nvfp4_status nvfp4_linear(const void *x, int64_t m, int64_t k, int64_t ldx, cons
 
 /* The whole layer for modules fused along N (e.g. q/k/v/gate projections
  * concatenated into one GEMM), each keeping its own weight global scale:
- * column j of segment i is scaled by s_x * seg_gscales[i] (paper §6).
+ * column j of segment i is scaled by s_x * seg_gscales[i] ("Why Gated DeltaNet
+ * Survives 4-Bit Quantization", §6 "Per-module calibration vs. fused-GEMM scaling").
  * seg_offsets host int64[nseg+1]; seg_gscales device float[nseg].
  * Errors: those of nvfp4_gemm for the GEMM's arguments and of
  * nvfp4_quantize_act for x, plus NVFP4_ERR_WORKSPACE for a NULL, unaligned or

@@ -140,7 +140,8 @@ def test_gemm_exact_on_representable_operands(nv):
 
 def test_fused_segments_match_separate_modules_and_collapsed_mode_fails(nv):
     """Per-segment epilogue == separate per-module GEMMs; the collapsed-max mode
-    (the serving mismatch of the paper's §6) mis-scales the smaller-scale module
+    (the serving mismatch of "Why Gated DeltaNet Survives 4-Bit Quantization",
+    §6 "Per-module calibration vs. fused-GEMM scaling") mis-scales the smaller-scale module
     by the scale ratio."""
     import torch
     m, k = 96, 512
