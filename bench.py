@@ -671,7 +671,7 @@ def fp4_peak_probe(nv, device_index=0):
     back from shared-memory-resident operands, no global-memory traffic, one CTA
     per SM).  Burst: launches of ~2 ms after an idle pause, median.  Sustained:
     launches of ~0.25 s back to back for >= 1 s, with the SM clock sampled.  The
-    same for the GEMM's per-stage scale-factor copies included."""
+    burst is also taken with the GEMM's per-stage scale-factor copies included."""
     import torch
     s = torch.cuda.current_stream()
 
@@ -692,6 +692,10 @@ def fp4_peak_probe(nv, device_index=0):
         for _ in range(7):
             time.sleep(0.05)
             burst.append(timed(burst_iters, copies))
+        tag = "with_scale_copies_" if copies else ""
+        out[f"{tag}burst_tflops"] = round(statistics.median(burst), 1)
+        if copies:
+            continue                                         # the sustained run is MMA-only
         sustained_iters = burst_iters * 125                  # ~0.25 s per launch
         sampler = ClockSampler(device_index)
         sampler.start()
@@ -705,8 +709,6 @@ def fp4_peak_probe(nv, device_index=0):
         torch.cuda.synchronize()
         clocks = sampler.stop()
         sec = e0.elapsed_time(e1) * 1e-3
-        tag = "with_scale_copies_" if copies else ""
-        out[f"{tag}burst_tflops"] = round(statistics.median(burst), 1)
         out[f"{tag}sustained_tflops"] = round(fl / sec / 1e12, 1)
         out[f"{tag}sustained_seconds"] = round(sec, 3)
         out[f"{tag}sustained_clocks"] = clocks
