@@ -264,7 +264,11 @@ __global__ void __launch_bounds__(THREADS, 2)
                 alpha = sx * p.s_w[seg];
             }
         }
-        if (mbar_wait_bounded(acc_full, 0, abort_flag, p.timeout_ns)) {
+        // The four warps agree on the outcome of their bounded waits before any of
+        // them reaches the named barrier below (a warp that gave up right at the
+        // deadline must not strand the others there).
+        const bool acc_ok = mbar_wait_bounded(acc_full, 0, abort_flag, p.timeout_ns);
+        if (!bar_red_or(2, 128, acc_ok ? 0u : 1u)) {
             tc_fence_after();
             // Every stage has landed and every MMA has read its operands, so the
             // stage buffers are free: the tile is staged there as [token][128
