@@ -307,3 +307,91 @@ def test_prefill_workload_sampled_rows(nv):
 def test_long_prefill_workload_sampled_rows(nv):
     wl = W.LONG_DOWN
     _workload_layer(nv, wl, wl.x(), rows=_rows_sample(wl.m, wl.cfg_id, 32)[::2])
+
+
+@pytest.mark.parametrize("m", [8, 40, 200], ids=["decode_T8", "decode_T64", "pair"])
+def test_inputs_rewritten_just_before_a_call_are_the_ones_it_reads(nv, m):
+    """Every GEMM is launched with programmatic stream serialization, so it may
+    start while the kernel before it still runs; the library's quantizers let
+    their dependents start early too.  Packed weights and activation codes
+    rewritten in place by the immediately preceding call (nothing in between on
+    the stream) must still be the ones the layer reads: the results equal those
+    computed from freshly allocated operands."""
+    import ctypes
+    import torch
+    n, k = 392, 1344
+    xb1, wb1, off = W.random_case(80 + m, m, n, k, seg_rows=[128, 264])
+    xb2, wb2, _ = W.random_case(90 + m, m, n, k, seg_rows=[128, 264])
+    x1, x2 = to_cuda_bf16(xb1), to_cuda_bf16(xb2)
+    w2 = to_cuda_bf16(wb2)
+    ref_pw = nv.pack_weight(w2, off)
+    expect_layer = nv.linear_fused(x1, ref_pw, flags=nv.FLAG_F32_OUT)
+    qx2, sfx2, sx2 = nv.quantize_act(x2)
+    expect_gemm = nv.gemm(qx2, sfx2, sx2, m, ref_pw, flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+
+    pw = nv.pack_weight(to_cuda_bf16(wb1), off)            # buffers that will be overwritten
+    qx, sfx, sx = nv.quantize_act(x1)
+    nv.linear_fused(x1, pw, flags=nv.FLAG_F32_OUT)          # warm, with the first weight
+    torch.cuda.synchronize()
+    L = nv.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    segs = (ctypes.c_int64 * len(off))(*off)
+    ws = torch.empty(nv.workspace_bytes(n, 0, k), dtype=torch.uint8, device="cuda")
+    ws_layer = torch.empty(nv.workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    # repack in place, then the layer right behind it
+    st = L.nvfp4_pack_weight(w2.data_ptr(), n, k, k, segs, len(off) - 1, None, pw.gscale.data_ptr(), pw.q.data_ptr(),
+                             pw.sf.data_ptr(), ws.data_ptr(), ws.numel(), stream)
+    assert st == nv.OK
+    y_layer = nv.linear_fused(x1, pw, flags=nv.FLAG_F32_OUT, ws=ws_layer)
+    # re-quantize the activations in place, then the GEMM right behind it
+    nv.quantize_act(x2, q=qx, sf=sfx, gscale_out=sx)
+    y_gemm = nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    assert torch.equal(y_layer, expect_layer)
+    assert torch.equal(y_gemm, expect_gemm)
+
+
+@pytest.mark.parametrize("m", [1, 32, 200], ids=["decode_T8", "decode_T32", "pair"])
+def test_layer_and_gemm_replay_from_a_cuda_graph(nv, m):
+    """The quantizer -> GEMM chain (with its programmatic launch edges) and the
+    stand-alone GEMM captured into one CUDA graph and replayed give the eager
+    results bit for bit, also when the inputs change between replays."""
+    import torch
+    n, k = 520, 1088
+    xb, wb, off = W.random_case(95 + m, m, n, k, seg_rows=[264, 256])
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    x = to_cuda_bf16(xb)
+    qx, sfx, sx = nv.quantize_act(x)
+    ws = torch.empty(nv.workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda")
+    y_layer = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    y_gemm = torch.empty((m, n), dtype=torch.float32, device="cuda")
+
+    def step():
+        nv.linear_fused(x, pw, out=y_layer, ws=ws)
+        nv.gemm(qx, sfx, sx, m, pw, out=y_gemm, flags=nv.FLAG_F32_OUT)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()                                           # first calls (per-device set-up) outside capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for seed in (96, 97):
+        xb2, _, _ = W.random_case(seed + m, m, n, k)
+        x.copy_(to_cuda_bf16(xb2))
+        q2, sf2, s2 = nv.quantize_act(x)
+        qx.copy_(q2)
+        sfx.copy_(sf2)
+        sx.copy_(s2)
+        g.replay()
+        torch.cuda.synchronize()
+        assert nv.get_device_error() == nv.OK
+        assert torch.equal(y_layer, nv.linear_fused(x, pw))
+        assert torch.equal(y_gemm, nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT))
+    del g
