@@ -92,6 +92,17 @@ typedef enum {
 #define NVFP4_FLAG_COLLAPSED_MAX_SCALE 0x2u  /* negative control: every column uses s_x * max(s_w),
                                                 the mismatch of "Why Gated DeltaNet Survives
                                                 4-Bit Quantization", §6; never for serving */
+#define NVFP4_FLAG_STATIC_WEIGHTS 0x4u       /* nvfp4_gemm: the caller guarantees that no work still
+                                                pending on the device writes the packed weight codes or
+                                                block scales (e.g. weights packed once at load time), so
+                                                the GEMM may request its first weight stages before it
+                                                waits for the preceding kernel in the stream to finish,
+                                                overlapping that kernel's end (activations, global
+                                                scales and the output are still touched only after the
+                                                wait).  Results are unchanged.  nvfp4_linear and
+                                                nvfp4_linear_fused accept it and always do this behind
+                                                their own quantizer.  A deployment option; no paper
+                                                counterpart. */
 #define NVFP4_FLAG_TEST_STALL 0x100u         /* testing only: the GEMM's producer withholds its second
                                                 K stage, so a bounded pipeline wait runs out; the call
                                                 writes no valid output and records NVFP4_ERR_TIMEOUT in

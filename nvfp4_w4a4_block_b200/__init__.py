@@ -41,6 +41,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 FLAG_F32_OUT = 0x1
 FLAG_COLLAPSED_MAX_SCALE = 0x2
+FLAG_STATIC_WEIGHTS = 0x4
 FLAG_TEST_STALL = 0x100
 FLAG_TEST_STALL_LATE = 0x200
 MAX_SEGMENTS = 8

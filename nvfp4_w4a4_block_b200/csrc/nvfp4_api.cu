@@ -489,24 +489,26 @@ nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s
 // GEMM + epilogue.  Up to 64 tokens take the swapped decode kernel, more take
 // the persistent CTA-pair kernel (256 x 256 tiles).  Both are launched with
 // programmatic stream serialization and touch no global memory before
-// griddepcontrol.wait, except that `early_weights` (set only when the preceding
-// kernel in the stream is this library's quantizer, whose early trigger comes
-// after all earlier work has completed) lets them request their first weight
-// stages before it.
+// griddepcontrol.wait, except that `early_weights` lets them request their
+// first weight stages before it.  It is set when the preceding kernel in the
+// stream is this library's quantizer (whose early trigger comes after all
+// earlier work has completed), or when the caller passed
+// NVFP4_FLAG_STATIC_WEIGHTS (no pending work writes the weights).
 nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
                          const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
-                         const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms, bool pdl,
+                         const float *seg_gscales, void *y, int64_t ldy, unsigned flags, int sms, bool early_weights,
                          cudaStream_t stream)
 {
+    const bool ew = early_weights;
     if (m <= 8)
-        return launch_decode<8>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
+        return launch_decode<8>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, ew, stream);
     if (m <= 16)
-        return launch_decode<16>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
+        return launch_decode<16>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, ew, stream);
     if (m <= 32)
-        return launch_decode<32>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
+        return launch_decode<32>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, ew, stream);
     if (m <= 64)
-        return launch_decode<64>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, pdl, stream);
-    return launch_pair(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, sms, pdl, stream);
+        return launch_decode<64>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, ew, stream);
+    return launch_pair(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, sms, ew, stream);
 }
 
 struct WorkspaceLayout {
@@ -529,8 +531,8 @@ nvfp4_status check_gemm_args(const uint8_t *qx, const uint8_t *sfx, const float 
 {
     if (m < 0 || n <= 0 || k <= 0)
         return NVFP4_ERR_INVALID_ARG;
-    if (flags & ~(NVFP4_FLAG_F32_OUT | NVFP4_FLAG_COLLAPSED_MAX_SCALE | NVFP4_FLAG_TEST_STALL |
-                  NVFP4_FLAG_TEST_STALL_LATE))
+    if (flags & ~(NVFP4_FLAG_F32_OUT | NVFP4_FLAG_COLLAPSED_MAX_SCALE | NVFP4_FLAG_STATIC_WEIGHTS |
+                  NVFP4_FLAG_TEST_STALL | NVFP4_FLAG_TEST_STALL_LATE))
         return NVFP4_ERR_INVALID_ARG;
     if (k % 64 != 0 || n % 8 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -657,8 +659,8 @@ nvfp4_status nvfp4_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x,
     int sms = 0;
     if ((st = device_setup(&sms)) != NVFP4_OK)
         return st;
-    return launch_gemm(qx, sfx, s_x, m, qw, sfw, n, k, ends, nseg, seg_gscales, y, ldy, flags, sms, false,
-                       reinterpret_cast<cudaStream_t>(stream));
+    return launch_gemm(qx, sfx, s_x, m, qw, sfw, n, k, ends, nseg, seg_gscales, y, ldy, flags, sms,
+                       (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 nvfp4_status nvfp4_linear_fused(const void *x, int64_t m, int64_t k, int64_t ldx, const float *act_gscale,

@@ -92,6 +92,7 @@ def test_gemm_validation(L):
     assert call(ldy=60) == nv.ERR_INVALID_ARG
     assert call(ldy=68) == nv.ERR_MISALIGNED
     assert call(flags=0x8) == nv.ERR_INVALID_ARG
+    assert call(flags=nv.FLAG_STATIC_WEIGHTS | nv.FLAG_F32_OUT, m=0, ldy=64) == nv.OK
     assert call(nseg=2) == nv.ERR_INVALID_ARG                       # NULL table needs nseg == 1
     assert call(seg=_segs(0, 32, 64), nseg=2, m=0) == nv.OK
     assert call(seg=_segs(0, 32, 60), nseg=2) == nv.ERR_INVALID_ARG  # last != N

@@ -395,3 +395,24 @@ def test_layer_and_gemm_replay_from_a_cuda_graph(nv, m):
         assert torch.equal(y_layer, nv.linear_fused(x, pw))
         assert torch.equal(y_gemm, nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT))
     del g
+
+
+@pytest.mark.parametrize("m", [8, 40, 200], ids=["decode_T8", "decode_T64", "pair"])
+def test_static_weights_flag_changes_nothing_but_the_launch_order(nv, m):
+    """With NVFP4_FLAG_STATIC_WEIGHTS the GEMM requests its first weight stages
+    before it waits for the preceding kernel; back-to-back calls on packed
+    (static) weights give the same bits as without the flag."""
+    import torch
+    xb, wb, off = W.random_case(98 + m, m, 520, 1344, seg_rows=[264, 256])
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    pw2 = nv.pack_weight(to_cuda_bf16(W.random_case(99 + m, m, 520, 1344, seg_rows=[264, 256])[1]), off)
+    qx, sfx, sx = nv.quantize_act(to_cuda_bf16(xb))
+    for flags in (0, nv.FLAG_F32_OUT):
+        ref1 = nv.gemm(qx, sfx, sx, m, pw, flags=flags)
+        ref2 = nv.gemm(qx, sfx, sx, m, pw2, flags=flags)
+        got = [nv.gemm(qx, sfx, sx, m, p, flags=flags | nv.FLAG_STATIC_WEIGHTS) for p in (pw, pw2, pw, pw2)]
+        torch.cuda.synchronize()
+        assert nv.get_device_error() == nv.OK
+        assert torch.equal(got[0], ref1) and torch.equal(got[2], ref1)
+        assert torch.equal(got[1], ref2) and torch.equal(got[3], ref2)
+
