@@ -423,7 +423,10 @@ def run_nvfp4(args, rank, world, local_rank):
             for c in range(copies):
                 nv.linear_fused(xs[m], pws[c], act_gscale=static, out=ym, ws=wss[m])
 
-        gg, gp, gc, gs = capture_graph(gemms), capture_graph(gemms_plain), capture_graph(calls), capture_graph(calls_static)
+        before = nv.launch_count()
+        gc = capture_graph(calls)
+        call_launches = (nv.launch_count() - before) // (2 * copies)
+        gg, gp, gs = capture_graph(gemms), capture_graph(gemms_plain), capture_graph(calls_static)
         tg = time_graph(gg, 20, copies)
         tp = time_graph(gp, 20, copies)
         tf = time_graph(gc, 20, copies)
@@ -436,6 +439,7 @@ def run_nvfp4(args, rank, world, local_rank):
                              gemm_no_static_flag_gbs=round(gb / (tp * 1e-3) / 1e9, 1),
                              call_us=round(tf * 1e3, 3), call_gbs=round(fb / (tf * 1e-3) / 1e9, 1),
                              call_static_scale_us=round(ts * 1e3, 3),
+                             call_launches=call_launches,
                              gemm_bytes=gb, call_bytes=fb)
     gm = per_m[str(mmax)]
     roofline = dict(bound="hbm", kernel="nvfp4_gemm_decode_kernel", workload=f"decode M={mmax}",
