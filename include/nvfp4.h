@@ -241,7 +241,8 @@ nvfp4_status nvfp4_linear_fused_noalloc(const void *x, int64_t m, int64_t k, int
  * sf           device block scales in the tensor-core layout (nvfp4_sf_bytes(rows, k)).
  * seg_offsets  host int64[nseg+1] row segments (NULL with nseg == 1).
  * seg_gscales  device float[nseg] global scale of each segment; they must be
- *              finite (a non-finite scale gives unspecified values).
+ *              finite and non-negative, as every global scale of the format is
+ *              (any other value gives unspecified values).
  * y            device bf16 [rows, k] with row stride ldy elements (16-byte aligned rows).
  * K % 64 == 0; any row count (rows == 0 is a no-op).  Needs no workspace. */
 nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t k,

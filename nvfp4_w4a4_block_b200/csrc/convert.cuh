@@ -112,17 +112,29 @@ __device__ __forceinline__ BlockTable block_table(float sd, float s)
     return t;
 }
 
+// PTX byte permute in its default mode: selector nibble n's low three bits pick
+// byte n of the result from {a (bytes 0..3), b (bytes 4..7)}; with the nibble's
+// bit 3 set the result byte is the picked byte's bit 7 replicated (0x00 / 0xFF).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
 // Four codes (nibbles 0..3 of `w`, element order) -> two words of bf16 pairs.
+// The high-byte table may carry the block scale's sign in bit 7 of every entry.
 __device__ __forceinline__ void expand4(const BlockTable &t, uint32_t w, uint32_t &out0, uint32_t &out1)
 {
     const uint32_t sel = w & 0x7777u;                          // magnitude indices
-    const uint32_t lo = __byte_perm(t.lo0, t.lo1, sel);        // low bytes of elements 0..3
-    const uint32_t hi = __byte_perm(t.hi0, t.hi1, sel);        // high bytes of elements 0..3
-    // sign bits: code bit 3 -> bf16 bit 15 of the element's half-word
-    const uint32_t s01 = ((w & 0x8u) << 12) | ((w & 0x80u) << 24);
-    const uint32_t s23 = ((w & 0x800u) << 4) | ((w & 0x8000u) << 16);
-    out0 = __byte_perm(lo, hi, 0x5140u) | s01;
-    out1 = __byte_perm(lo, hi, 0x7362u) | s23;
+    const uint32_t lo = prmt(t.lo0, t.lo1, sel);               // low bytes of elements 0..3
+    // Code signs (bit 3 of each nibble) as bit 7 of element bytes 0..3: the
+    // sign-replicating picks read codes 0 and 2 from w << 4 (their sign bits at 7
+    // and 15) and codes 1 and 3 from w itself (at 7 and 15).
+    const uint32_t sg = prmt(w << 4, w, 0xD9C8u) & 0x80808080u;
+    const uint32_t hi = prmt(t.hi0, t.hi1, sel) ^ sg;          // high bytes of elements 0..3
+    out0 = prmt(lo, hi, 0x5140u);
+    out1 = prmt(lo, hi, 0x7362u);
 }
 
 // ------------------------------------------------------------------ expansion
@@ -201,15 +213,13 @@ __global__ void __launch_bounds__(kThreads) expand_kernel(ExpandParams p)
                 ++seg;
             const uint32_t sb = (sfv[j] >> (8 * (g >> 1))) & 0xFFu;
             const uint4 tv = s_lut[seg * 128 + (sb & 0x7Fu)];
-            const BlockTable tb = {tv.x, tv.y, tv.z, tv.w};
-            const uint32_t neg = (sb & 0x80u) ? 0x80008000u : 0u;
+            // A scale byte with its sign bit set negates the block: flip bit 7 of
+            // every high-byte table entry once instead of every output element.
+            const uint32_t neg = (sb & 0x80u) ? 0x80808080u : 0u;
+            const BlockTable tb = {tv.x, tv.y, tv.z ^ neg, tv.w ^ neg};
             uint4 o;
             expand4(tb, cur[j], o.x, o.y);
             expand4(tb, cur[j] >> 16, o.z, o.w);
-            o.x ^= neg;
-            o.y ^= neg;
-            o.z ^= neg;
-            o.w ^= neg;
             *reinterpret_cast<uint4 *>(out) = o;
             out += 32 * p.ldy;
         }
