@@ -457,7 +457,7 @@ def run_nvfp4(args, rank, world, local_rank):
     # host buffers alternate between two sets, and a set is refilled only after the
     # copies that read it have completed, so every step's inputs and results really
     # cross PCIe inside the timed region.
-    E2E_STEPS = 4                         # steps per captured graph
+    E2E_STEPS = 8                         # steps per captured graph (one pipeline fill and drain each)
     order = sorted(ms, reverse=True)
     rows_at, r0 = {}, 0
     for m in order:                       # the step's inputs (and results) as one block of rows
