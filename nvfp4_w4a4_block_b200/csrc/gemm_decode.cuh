@@ -1,4 +1,4 @@
-// gemm_decode.cuh -- block-scaled FP4 GEMM for few tokens (M <= 64), sm_100a.
+// gemm_decode.cuh -- block-scaled FP4 GEMM for few tokens (M <= 128), sm_100a.
 //
 // Same product and epilogue as gemm_pair.cuh ("Why Gated DeltaNet Survives 4-Bit
 // Quantization", §2 "NVFP4"; per-module global scales of §6), organised for the
@@ -7,7 +7,7 @@
 //
 //   * Operands are swapped: the weight tile (128 rows of N) is the MMA's A operand,
 //     so it fills the 128 tensor-memory lanes, and the tokens are the MMA's N
-//     (T = 8, 16, 32 or 64).  No tile carries zero padding of the token dimension
+//     (T = 8, 16, 32, 64 or 128).  No tile carries zero padding of the token dimension
 //     beyond T, and a stage is ~22-28 KB instead of 54 KB.
 //   * One CTA owns one 128-row weight tile over the whole K; two CTAs fit on an SM,
 //     so N/128 tiles (272 for N = 34816) are all resident at once and each SM keeps
@@ -22,7 +22,7 @@
 //
 // Roles: warp 0 producer (TMA + bulk copies), warp 1 MMA issuer (one elected lane),
 // warps 2..5 epilogue (tcgen05.ld of the 128 x T accumulator, x alpha(n), the tile
-// staged as [token][128 columns] in the idle stage buffers, then 16-byte stores
+// staged as [token][128 columns] in the idle stage buffers (weights and tokens), then 16-byte stores
 // along each token's row of Y).
 #pragma once
 
@@ -69,11 +69,15 @@ struct Cfg {
     static constexpr int SMEM_ALLOC = OFF_MISC + 64 + 1024;
     static constexpr int TMEM_SFA = T;                 // columns after the accumulator
     static constexpr int TMEM_SFB = T + KB * 4;
-    static constexpr int TMEM_COLS = (T + KB * 8 <= 32) ? 32 : (T + KB * 8 <= 64) ? 64 : 128;
+    static constexpr int TMEM_COLS = (T + KB * 8 <= 32)    ? 32
+                                     : (T + KB * 8 <= 64)  ? 64
+                                     : (T + KB * 8 <= 128) ? 128
+                                                           : 256;   // two CTAs per SM: at most 256 each
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(SMEM_ALLOC <= SMEM_LIMIT, "two CTAs per SM");
     static_assert(B_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
-    static_assert(STAGES * A_BYTES >= T * BW * 4, "the epilogue stages a fp32 tile in the weight buffers");
+    static_assert(OFF_SFA >= T * BW * 4, "the epilogue stages a fp32 tile in the operand buffers");
+    static_assert(TMEM_COLS <= 256, "two CTAs per SM share the 512 tensor-memory columns");
 };
 
 struct Params {

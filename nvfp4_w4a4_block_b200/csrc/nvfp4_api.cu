@@ -157,6 +157,8 @@ nvfp4_status device_setup(int *sms)
                                  decode::Cfg<32>::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Cfg<64>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Cfg<128>::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(peak::mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  peak::SMEM_ALLOC) != cudaSuccess)
             return NVFP4_ERR_CUDA;
@@ -486,7 +488,7 @@ nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s
                               stream, true, tw, tx, p));
 }
 
-// GEMM + epilogue.  Up to 64 tokens take the swapped decode kernel, more take
+// GEMM + epilogue.  Up to 128 tokens take the swapped decode kernel, more take
 // the persistent CTA-pair kernel (256 x 256 tiles).  Both are launched with
 // programmatic stream serialization and touch no global memory before
 // griddepcontrol.wait, except that `early_weights` lets them request their
@@ -508,6 +510,12 @@ nvfp4_status launch_gemm(const uint8_t *qx, const uint8_t *sfx, const float *s_x
         return launch_decode<32>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, ew, stream);
     if (m <= 64)
         return launch_decode<64>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, ew, stream);
+    // 65..128 tokens: the weight stream still bounds the GEMM, which the swapped
+    // kernel serves better than 256-row pair tiles (N = 34816, K = 5120: M = 128
+    // measured 25.3 us on the pair kernel).
+    if (m <= 128)
+        return launch_decode<128>(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, ew,
+                                  stream);
     return launch_pair(qx, sfx, s_x, m, qw, sfw, n, k, seg_ends, nseg, seg_gscales, y, ldy, flags, sms, ew, stream);
 }
 

@@ -99,10 +99,10 @@ def test_gemm_eight_modules_some_eight_columns_wide(nv, m):
     assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), bf16_rne_from_f32(y32.cpu().numpy()))
 
 
-@pytest.mark.parametrize("m", [1, 7, 8, 9, 16, 17, 31, 32, 33, 63, 64, 65])
+@pytest.mark.parametrize("m", [1, 7, 8, 9, 16, 17, 31, 32, 33, 63, 64, 65, 100, 128, 129])
 def test_gemm_token_buckets(nv, m):
-    """Every token-count bucket of the swapped decode kernel (8/16/32/64) and the
-    switch to the tile kernel above 64, with ragged N (200 = 128 + 72) and a
+    """Every token-count bucket of the swapped decode kernel (8/16/32/64/128) and
+    the switch to the tile kernel above 128, with ragged N (200 = 128 + 72) and a
     partial last K stage (320 = 256 + 64), two segments."""
     import torch
     xb, wb, off = W.random_case(20 + m, m, 200, 320, seg_rows=[64, 136])
