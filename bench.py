@@ -953,6 +953,7 @@ def _prof_mma_peak(launches):
 PROFILE_CASES = {
     "mma_peak": _prof_mma_peak,
     "gemm_decode_m32": lambda L: _prof_gemm(32, 34816, 5120, [0, 17408, 34816], L),
+    "gemm_decode_m128": lambda L: _prof_gemm(128, 34816, 5120, [0, 17408, 34816], L),
     "gemm_prefill_8192x17408x5120": lambda L: _prof_gemm(8192, 17408, 5120, [0, 17408], L, "student_t3"),
     "gemm_long_32768x5120x17408": lambda L: _prof_gemm(32768, 5120, 17408, [0, 5120], L),
     "quantize_32768x17408_static": lambda L: _prof_quantize(32768, 17408, L, True),
