@@ -48,6 +48,7 @@ struct DeviceInfo {
     int tile_quant_ctas_per_sm = 1;
     int expand_ctas_per_sm = 1;
     bool cluster_quant = false;     // a 16-CTA cluster of the decode quantizer can be resident
+    bool cluster_quant_large = false;   // ... of its 12-unit instance
 };
 
 std::mutex g_mu;
@@ -55,10 +56,13 @@ DeviceInfo g_dev[64];
 thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
 thread_local int g_expand_ctas = 148;       // resident expansion CTAs on the current device
 thread_local bool g_cluster_quant = false;  // decode quantizer cluster available on the current device
+thread_local bool g_cluster_quant_large = false;  // its 12-unit instance too
 constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder below, tiled encoder above
 // Decode-sized activations: one cluster launch holds the whole tensor in
-// registers (quantize_cluster_kernel) up to this many elements.
-constexpr int64_t kClusterQuantElems = int64_t(kClusterCtas) * kClusterThreads * kClusterUnits * 8;
+// registers (quantize_cluster_kernel) up to this many elements, with 5 or with
+// 12 units per thread.
+constexpr int64_t kClusterQuantElems = int64_t(kClusterCtas) * kClusterThreads * kClusterUnitsSmall * 8;
+constexpr int64_t kClusterQuantElemsLarge = int64_t(kClusterCtas) * kClusterThreads * kClusterUnitsLarge * 8;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
 PFN_cuCtxGetId_v12000 g_ctx_get_id = nullptr;
@@ -172,8 +176,10 @@ nvfp4_status device_setup(int *sms)
         }
         // The decode-size quantizer runs as one cluster of 16 CTAs (beyond the
         // portable 8, which sm_100 allows once the kernel opts in).
-        if (cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(quantize_cluster_kernel<kClusterUnitsSmall>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+            cudaFuncSetAttribute(quantize_cluster_kernel<kClusterUnitsLarge>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         {
             // A device (or partition) that cannot hold one such cluster takes the
@@ -182,14 +188,22 @@ nvfp4_status device_setup(int *sms)
             cc.gridDim = dim3(kClusterCtas);
             cc.blockDim = dim3(kClusterThreads);
             int nclusters = 0;
-            d.cluster_quant = cudaOccupancyMaxActiveClusters(&nclusters, quantize_cluster_kernel, &cc) == cudaSuccess &&
+            d.cluster_quant = cudaOccupancyMaxActiveClusters(&nclusters, quantize_cluster_kernel<kClusterUnitsSmall>,
+                                                             &cc) == cudaSuccess &&
                               nclusters >= 1;
             cudaGetLastError();     // a refused query leaves no sticky error behind
+            nclusters = 0;
+            d.cluster_quant_large = d.cluster_quant &&
+                                    cudaOccupancyMaxActiveClusters(&nclusters,
+                                                                   quantize_cluster_kernel<kClusterUnitsLarge>, &cc) ==
+                                        cudaSuccess &&
+                                    nclusters >= 1;
+            cudaGetLastError();
             // NVFP4_NO_CLUSTER_QUANTIZER=1 takes the same fallback on any device
             // (it is how the fallback is tested on parts where the cluster fits).
             const char *no_cluster = std::getenv("NVFP4_NO_CLUSTER_QUANTIZER");
             if (no_cluster != nullptr && no_cluster[0] == '1')
-                d.cluster_quant = false;
+                d.cluster_quant = d.cluster_quant_large = false;
         }
         int occ = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_tile_kernel, kQuantThreads, 0) !=
@@ -209,6 +223,7 @@ nvfp4_status device_setup(int *sms)
     g_tile_quant_ctas = d.sms * d.tile_quant_ctas_per_sm;
     g_expand_ctas = d.sms * d.expand_ctas_per_sm;
     g_cluster_quant = d.cluster_quant;
+    g_cluster_quant_large = d.cluster_quant_large;
     return d.status;
 }
 
@@ -273,16 +288,19 @@ int quant_grid(int sms, int64_t rows, int64_t k)
 }
 
 // Quantization of [rows, k] (rows split into segments).  One segment, at most
-// 327680 elements (decode): one cluster launch reduces the amax (dynamic scale)
-// and encodes.  Up to 2^20 elements: the per-unit encoder, after an amax pass in
-// dynamic mode.  Larger (or several segments): amax passes and the tiled encoder.
+// 786432 elements (decode, up to 153 tokens at K = 5120): one cluster launch
+// reduces the amax (dynamic scale) and encodes, with 5 units per thread up to
+// 327680 elements and 12 above.  Up to 2^20 elements: the per-unit encoder,
+// after an amax pass in dynamic mode.  Larger (or several segments): amax passes
+// and the tiled encoder.
 nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx, const int64_t *seg_ends, int nseg,
                              const float *static_scale, float *scale_out, uint8_t *q, uint8_t *sf,
                              uint32_t *partials, int sms, cudaStream_t stream)
 {
     const int ga = amax_grid(sms, rows, k);
     if (nseg == 1 && rows * k <= kSmallQuantElems) {
-        const bool cluster = g_cluster_quant && rows * k <= kClusterQuantElems;
+        const bool cluster_small = g_cluster_quant && rows * k <= kClusterQuantElems;
+        const bool cluster = cluster_small || (g_cluster_quant_large && rows * k <= kClusterQuantElemsLarge);
         if (static_scale == nullptr && !cluster) {
             AmaxParams ap;
             ap.x = static_cast<const uint16_t *>(x);
@@ -311,8 +329,12 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
         qp.npartial = ga;
         qp.scale_out = scale_out;
         qp.timeout_ns = g_timeout_ns.load();
+        if (cluster_small)
+            return cuda_status(launch(quantize_cluster_kernel<kClusterUnitsSmall>, kClusterCtas, kClusterThreads, 0,
+                                      stream, true, qp));
         if (cluster)
-            return cuda_status(launch(quantize_cluster_kernel, kClusterCtas, kClusterThreads, 0, stream, true, qp));
+            return cuda_status(launch(quantize_cluster_kernel<kClusterUnitsLarge>, kClusterCtas, kClusterThreads, 0,
+                                      stream, true, qp));
         const int grid = quant_grid(sms, rows, k);
         return cuda_status(launch(quantize_kernel, grid, kQuantThreads, 0, stream, true, qp));
     }

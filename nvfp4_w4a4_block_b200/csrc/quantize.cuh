@@ -326,15 +326,21 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
 
 // Decode-sized activations in one launch: a cluster of kClusterCtas CTAs (16:
 // a non-portable cluster size the launcher opts into) holds the whole tensor in
-// registers (at most kClusterUnits 16-byte units per thread), reduces the
+// registers (at most UNITS 16-byte units per thread), reduces the
 // absolute maximum over the cluster through distributed shared memory when the
 // scale is dynamic, and encodes from the same registers -- one read of X, no
 // amax pass, no workspace.  Unit-to-lane mapping, arithmetic and stores are
 // those of quantize_kernel.
+// Two instances: 5 units per thread (up to 327680 elements, 63 registers, so a
+// CTA of it fits beside the two decode GEMM CTAs still running on an SM when it
+// starts) and 12 units (up to 786432 elements, e.g. 65-128 tokens at K = 5120;
+// 127 registers, the whole register file of an SM).
 constexpr int kClusterCtas = 16;
 constexpr int kClusterThreads = 512;
-constexpr int kClusterUnits = 5;
+constexpr int kClusterUnitsSmall = 5;
+constexpr int kClusterUnitsLarge = 12;
 
+template <int UNITS>
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
     quantize_cluster_kernel(QuantParams p)
 {
@@ -375,14 +381,14 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     const int64_t gtid = static_cast<int64_t>(rank) * kClusterThreads + threadIdx.x;
     // Unit j of this thread is gtid + j * nthreads; its (row, column) advance by a
     // fixed step, so only the first needs a division.
-    // The launch covers at most kClusterCtas * kClusterThreads * kClusterUnits
+    // The launch covers at most kClusterCtas * kClusterThreads * UNITS
     // units, so a unit's row and column fit in 32 bits.
     const int step_r = static_cast<int>(nthreads / upr), step_c = static_cast<int>(nthreads % upr);
-    int row[kClusterUnits], col[kClusterUnits];
+    int row[UNITS], col[UNITS];
     row[0] = static_cast<int>(gtid / upr);
     col[0] = static_cast<int>(gtid % upr);
 #pragma unroll
-    for (int j = 1; j < kClusterUnits; ++j) {
+    for (int j = 1; j < UNITS; ++j) {
         row[j] = row[j - 1] + step_r;
         col[j] = col[j - 1] + step_c;
         if (col[j] >= upr) {
@@ -390,10 +396,10 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
             ++row[j];
         }
     }
-    uint4 v[kClusterUnits];
+    uint4 v[UNITS];
     uint32_t b = 0;
 #pragma unroll
-    for (int j = 0; j < kClusterUnits; ++j) {
+    for (int j = 0; j < UNITS; ++j) {
         v[j] = row[j] < p.rows ? __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(row[j]) * p.ldx +
                                                                     col[j] * 8))
                                : make_uint4(0, 0, 0, 0);
@@ -453,7 +459,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     const float s = s_sc[0], dg = s_sc[1];
 
 #pragma unroll
-    for (int j = 0; j < kClusterUnits; ++j) {
+    for (int j = 0; j < UNITS; ++j) {
         const int64_t u = gtid + j * nthreads;
         if (__shfl_sync(0xFFFFFFFFu, u, 0) >= total)       // warp-uniform: lane 0 holds the warp's first unit
             break;

@@ -185,15 +185,33 @@ def test_quantize_nonfinite_sets_device_error(nv):
     assert nv.get_device_error() == nv.OK
 
 
-@pytest.mark.parametrize("m,k", [(1, 5120), (4, 5120), (8, 5120), (9, 5120), (1, 40960), (1, 41024), (2, 20480),
-                                 (32, 5120), (38, 5120), (39, 5120), (64, 5120),
-                                 (65, 5120), (18, 17408), (19, 17408), (1, 196608), (1, 327680), (1, 327744)])
-def test_quantize_decode_sizes_around_the_one_launch_limit(nv, m, k):
-    """Dynamic-scale activations up to 327680 elements are quantized in one
-    cluster launch (the whole tensor held in registers); just above that the
-    amax pass and the per-unit encoder take over.  Both sides of the limit, and
-    shapes whose pad rows fill most of the scale block."""
+# (m, k, launches of a dynamic-scale quantization): one cluster launch up to
+# 327680 elements (5 units per thread) and up to 786432 (its 12-unit instance);
+# above that the amax pass and the per-unit encoder (two launches).
+ONE_LAUNCH_LIMIT_CASES = [
+    (1, 5120, 1), (4, 5120, 1), (8, 5120, 1), (9, 5120, 1), (1, 40960, 1), (1, 41024, 1), (2, 20480, 1),
+    (32, 5120, 1), (38, 5120, 1), (39, 5120, 1), (64, 5120, 1), (18, 17408, 1), (19, 17408, 1),
+    (1, 196608, 1), (1, 327680, 1), (1, 327744, 1),
+    (65, 5120, 1), (100, 5120, 1), (128, 5120, 1), (153, 5120, 1), (154, 5120, 2),
+    (45, 17408, 1), (46, 17408, 2), (1, 786432, 1), (1, 786496, 2),
+]
+
+
+@pytest.mark.parametrize("m,k,launches", ONE_LAUNCH_LIMIT_CASES)
+def test_quantize_decode_sizes_around_the_one_launch_limit(nv, m, k, launches):
+    """Dynamic-scale activations are quantized in one cluster launch (the whole
+    tensor held in registers) up to 327680 elements with 5 units per thread and
+    up to 786432 with 12; just above that the amax pass and the per-unit encoder
+    take over.  Both sides of each limit, and shapes whose pad rows fill most of
+    the scale block."""
+    import torch
     x, _, _ = W.random_case(33, m, 8, k)
+    xt = to_cuda_bf16(x)
+    torch.cuda.synchronize()
+    c0 = nv.launch_count()
+    nv.quantize_act(xt)
+    torch.cuda.synchronize()
+    assert nv.launch_count() - c0 == launches
     _compare(nv, x)
 
 
