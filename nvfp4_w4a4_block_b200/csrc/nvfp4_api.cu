@@ -48,6 +48,7 @@ struct DeviceInfo {
     int tile_quant_ctas_per_sm = 1;
     int expand_ctas_per_sm = 1;
     bool cluster_quant = false;     // a 16-CTA cluster of the decode quantizer can be resident
+    bool cluster_quant_mid = false;     // ... of its 1024-thread instance
     bool cluster_quant_large = false;   // ... of its 12-unit instance
 };
 
@@ -56,13 +57,18 @@ DeviceInfo g_dev[64];
 thread_local int g_tile_quant_ctas = 148;   // resident tile-quantize CTAs on the current device
 thread_local int g_expand_ctas = 148;       // resident expansion CTAs on the current device
 thread_local bool g_cluster_quant = false;  // decode quantizer cluster available on the current device
+thread_local bool g_cluster_quant_mid = false;    // its 1024-thread instance too
 thread_local bool g_cluster_quant_large = false;  // its 12-unit instance too
 constexpr int64_t kSmallQuantElems = int64_t(1) << 20;   // per-unit encoder below, tiled encoder above
 // Decode-sized activations: one cluster launch holds the whole tensor in
-// registers (quantize_cluster_kernel) up to this many elements, with 5 or with
-// 12 units per thread.
-constexpr int64_t kClusterQuantElems = int64_t(kClusterCtas) * kClusterThreads * kClusterUnitsSmall * 8;
-constexpr int64_t kClusterQuantElemsLarge = int64_t(kClusterCtas) * kClusterThreads * kClusterUnitsLarge * 8;
+// registers (quantize_cluster_kernel) up to these many elements (5 units x 512
+// threads, 5 x 1024, 12 x 512 per CTA).
+#define NVFP4_CLUSTER_SMALL quantize_cluster_kernel<5, 512>
+#define NVFP4_CLUSTER_MID quantize_cluster_kernel<5, 1024>
+#define NVFP4_CLUSTER_LARGE quantize_cluster_kernel<12, 512>
+constexpr int64_t kClusterQuantElems = int64_t(kClusterCtas) * 512 * 5 * 8;
+constexpr int64_t kClusterQuantElemsMid = int64_t(kClusterCtas) * 1024 * 5 * 8;
+constexpr int64_t kClusterQuantElemsLarge = int64_t(kClusterCtas) * 512 * 12 * 8;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
 PFN_cuCtxGetId_v12000 g_ctx_get_id = nullptr;
@@ -176,34 +182,32 @@ nvfp4_status device_setup(int *sms)
         }
         // The decode-size quantizer runs as one cluster of 16 CTAs (beyond the
         // portable 8, which sm_100 allows once the kernel opts in).
-        if (cudaFuncSetAttribute(quantize_cluster_kernel<kClusterUnitsSmall>,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
-            cudaFuncSetAttribute(quantize_cluster_kernel<kClusterUnitsLarge>,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        if (cudaFuncSetAttribute(NVFP4_CLUSTER_SMALL, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(NVFP4_CLUSTER_MID, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+            cudaFuncSetAttribute(NVFP4_CLUSTER_LARGE, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess)
             return NVFP4_ERR_CUDA;
         {
             // A device (or partition) that cannot hold one such cluster takes the
             // amax pass + per-unit encoder instead.
-            cudaLaunchConfig_t cc = {};
-            cc.gridDim = dim3(kClusterCtas);
-            cc.blockDim = dim3(kClusterThreads);
-            int nclusters = 0;
-            d.cluster_quant = cudaOccupancyMaxActiveClusters(&nclusters, quantize_cluster_kernel<kClusterUnitsSmall>,
-                                                             &cc) == cudaSuccess &&
-                              nclusters >= 1;
-            cudaGetLastError();     // a refused query leaves no sticky error behind
-            nclusters = 0;
-            d.cluster_quant_large = d.cluster_quant &&
-                                    cudaOccupancyMaxActiveClusters(&nclusters,
-                                                                   quantize_cluster_kernel<kClusterUnitsLarge>, &cc) ==
-                                        cudaSuccess &&
-                                    nclusters >= 1;
-            cudaGetLastError();
+            auto resident = [](auto kernel, int threads) {
+                cudaLaunchConfig_t cc = {};
+                cc.gridDim = dim3(kClusterCtas);
+                cc.blockDim = dim3(static_cast<unsigned>(threads));
+                int nclusters = 0;
+                const bool ok = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cc) == cudaSuccess && nclusters >= 1;
+                cudaGetLastError();     // a refused query leaves no sticky error behind
+                return ok;
+            };
+            d.cluster_quant = resident(NVFP4_CLUSTER_SMALL, 512);
+            d.cluster_quant_mid = d.cluster_quant && resident(NVFP4_CLUSTER_MID, 1024);
+            d.cluster_quant_large = d.cluster_quant && resident(NVFP4_CLUSTER_LARGE, 512);
             // NVFP4_NO_CLUSTER_QUANTIZER=1 takes the same fallback on any device
             // (it is how the fallback is tested on parts where the cluster fits).
             const char *no_cluster = std::getenv("NVFP4_NO_CLUSTER_QUANTIZER");
             if (no_cluster != nullptr && no_cluster[0] == '1')
-                d.cluster_quant = d.cluster_quant_large = false;
+                d.cluster_quant = d.cluster_quant_mid = d.cluster_quant_large = false;
         }
         int occ = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_tile_kernel, kQuantThreads, 0) !=
@@ -223,6 +227,7 @@ nvfp4_status device_setup(int *sms)
     g_tile_quant_ctas = d.sms * d.tile_quant_ctas_per_sm;
     g_expand_ctas = d.sms * d.expand_ctas_per_sm;
     g_cluster_quant = d.cluster_quant;
+    g_cluster_quant_mid = d.cluster_quant_mid;
     g_cluster_quant_large = d.cluster_quant_large;
     return d.status;
 }
@@ -289,8 +294,9 @@ int quant_grid(int sms, int64_t rows, int64_t k)
 
 // Quantization of [rows, k] (rows split into segments).  One segment, at most
 // 786432 elements (decode, up to 153 tokens at K = 5120): one cluster launch
-// reduces the amax (dynamic scale) and encodes, with 5 units per thread up to
-// 327680 elements and 12 above.  Up to 2^20 elements: the per-unit encoder,
+// reduces the amax (dynamic scale) and encodes: 512 threads x 5 units per CTA up
+// to 327680 elements, 1024 x 5 up to 655360 (measured 0.3-0.9 us faster per call
+// than 512 x 12 at 65-128 tokens), 512 x 12 above.  Up to 2^20 elements: the per-unit encoder,
 // after an amax pass in dynamic mode.  Larger (or several segments): amax passes
 // and the tiled encoder.
 nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx, const int64_t *seg_ends, int nseg,
@@ -299,8 +305,12 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
 {
     const int ga = amax_grid(sms, rows, k);
     if (nseg == 1 && rows * k <= kSmallQuantElems) {
-        const bool cluster_small = g_cluster_quant && rows * k <= kClusterQuantElems;
-        const bool cluster = cluster_small || (g_cluster_quant_large && rows * k <= kClusterQuantElemsLarge);
+        const int64_t elems = rows * k;
+        const bool cluster_small = g_cluster_quant && elems <= kClusterQuantElems;
+        const bool cluster_mid = !cluster_small && g_cluster_quant_mid && elems <= kClusterQuantElemsMid;
+        const bool cluster_large = !cluster_small && !cluster_mid && g_cluster_quant_large &&
+                                   elems <= kClusterQuantElemsLarge;
+        const bool cluster = cluster_small || cluster_mid || cluster_large;
         if (static_scale == nullptr && !cluster) {
             AmaxParams ap;
             ap.x = static_cast<const uint16_t *>(x);
@@ -330,11 +340,11 @@ nvfp4_status launch_quantize(const void *x, int64_t rows, int64_t k, int64_t ldx
         qp.scale_out = scale_out;
         qp.timeout_ns = g_timeout_ns.load();
         if (cluster_small)
-            return cuda_status(launch(quantize_cluster_kernel<kClusterUnitsSmall>, kClusterCtas, kClusterThreads, 0,
-                                      stream, true, qp));
-        if (cluster)
-            return cuda_status(launch(quantize_cluster_kernel<kClusterUnitsLarge>, kClusterCtas, kClusterThreads, 0,
-                                      stream, true, qp));
+            return cuda_status(launch(NVFP4_CLUSTER_SMALL, kClusterCtas, 512, 0, stream, true, qp));
+        if (cluster_mid)
+            return cuda_status(launch(NVFP4_CLUSTER_MID, kClusterCtas, 1024, 0, stream, true, qp));
+        if (cluster_large)
+            return cuda_status(launch(NVFP4_CLUSTER_LARGE, kClusterCtas, 512, 0, stream, true, qp));
         const int grid = quant_grid(sms, rows, k);
         return cuda_status(launch(quantize_kernel, grid, kQuantThreads, 0, stream, true, qp));
     }

@@ -331,20 +331,20 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p)
 // scale is dynamic, and encodes from the same registers -- one read of X, no
 // amax pass, no workspace.  Unit-to-lane mapping, arithmetic and stores are
 // those of quantize_kernel.
-// Two instances: 5 units per thread (up to 327680 elements, 63 registers, so a
-// CTA of it fits beside the two decode GEMM CTAs still running on an SM when it
-// starts) and 12 units (up to 786432 elements, e.g. 65-128 tokens at K = 5120;
-// 127 registers, the whole register file of an SM).
+// Instances (units per thread x threads per CTA):
+//   5 x 512   up to 327680 elements; 63 registers, so that a CTA fits beside the
+//             two decode GEMM CTAs still running on an SM when it starts;
+//   5 x 1024  up to 655360 elements (128 tokens at K = 5120), half the serial
+//             work per thread of 10 x 512; a whole register file per CTA;
+//   12 x 512  up to 786432 elements; 127 registers, a whole register file.
 constexpr int kClusterCtas = 16;
 constexpr int kClusterThreads = 512;
-constexpr int kClusterUnitsSmall = 5;
-constexpr int kClusterUnitsLarge = 12;
 
-template <int UNITS>
-__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
+template <int UNITS, int THREADS>
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(THREADS)
     quantize_cluster_kernel(QuantParams p)
 {
-    __shared__ uint32_t s_red[kClusterThreads / 32];
+    __shared__ uint32_t s_red[THREADS / 32];
     __shared__ uint32_t s_peer_max[kClusterCtas];        // entry r: CTA r's maximum, pushed by CTA r
     __shared__ __align__(8) uint64_t s_pushes;           // completes when all kClusterCtas entries landed
     __shared__ float s_sc[2];
@@ -377,11 +377,11 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
 
     const int64_t upr = p.k >> 3;
     const int64_t total = p.rows * upr;
-    const int64_t nthreads = static_cast<int64_t>(kClusterCtas) * kClusterThreads;
-    const int64_t gtid = static_cast<int64_t>(rank) * kClusterThreads + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(kClusterCtas) * THREADS;
+    const int64_t gtid = static_cast<int64_t>(rank) * THREADS + threadIdx.x;
     // Unit j of this thread is gtid + j * nthreads; its (row, column) advance by a
     // fixed step, so only the first needs a division.
-    // The launch covers at most kClusterCtas * kClusterThreads * UNITS
+    // The launch covers at most kClusterCtas * THREADS * UNITS
     // units, so a unit's row and column fit in 32 bits.
     const int step_r = static_cast<int>(nthreads / upr), step_c = static_cast<int>(nthreads % upr);
     int row[UNITS], col[UNITS];
@@ -414,7 +414,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
         __syncthreads();
         cluster_wait_acquire();                          // every CTA's s_pushes is initialised
         if (threadIdx.x < 32) {
-            uint32_t m = lane < kClusterThreads / 32 ? s_red[lane] : 0u;
+            uint32_t m = lane < THREADS / 32 ? s_red[lane] : 0u;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
