@@ -20,6 +20,7 @@
 #include "nvfp4.h"
 #include "convert.cuh"
 #include "gemm_decode.cuh"
+#include "gemm_decode_split.cuh"
 #include "gemm_pair.cuh"
 #include "mma_peak.cuh"
 #include "quantize.cuh"
@@ -169,6 +170,12 @@ nvfp4_status device_setup(int *sms)
                                  decode::Cfg<64>::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Cfg<128>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::nvfp4_gemm_decode_split_kernel<8>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, decode::SplitCfg<8>::SMEM_ALLOC) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(decode::nvfp4_gemm_decode_split_kernel<16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, decode::SplitCfg<16>::SMEM_ALLOC) !=
+                cudaSuccess ||
             cudaFuncSetAttribute(peak::mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  peak::SMEM_ALLOC) != cudaSuccess)
             return NVFP4_ERR_CUDA;
@@ -481,6 +488,10 @@ nvfp4_status launch_pair(const uint8_t *qx, const uint8_t *sfx, const float *s_x
                               pair::SMEM_ALLOC, stream, true, ta, tb, tsa, tsb, ty, p));
 }
 
+// The split decode kernel serves up to this many weight tiles times two (one
+// tile per two SMs of a B200's 148).
+constexpr int kSplitMaxTilesTimes2 = 148;
+
 template <int T>
 nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s_x, int64_t m, const uint8_t *qw,
                            const uint8_t *sfw, int64_t n, int64_t k, const int64_t *seg_ends, int nseg,
@@ -516,6 +527,17 @@ nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s
     p.stall_stage = (flags & NVFP4_FLAG_TEST_STALL) ? 1 : (flags & NVFP4_FLAG_TEST_STALL_LATE) ? p.k_stages - 1 : -1;
     p.early_weights = early_weights ? 1 : 0;
     const int grid = static_cast<int>((n + decode::BW - 1) / decode::BW);
+    if constexpr (T <= 16) {
+        // Few weight tiles (at most one per two SMs) and a K of at least 8
+        // stages: each tile runs on a cluster of decode::kSplit CTAs, one K
+        // range each (gemm_decode_split.cuh).
+        if (grid * 2 <= kSplitMaxTilesTimes2 && p.k_stages >= 2 * decode::kSplit) {
+            if (flags & NVFP4_FLAG_TEST_STALL_LATE)          // the last stage of each CTA's K range
+                p.stall_stage = p.k_stages / decode::kSplit - 1;
+            return cuda_status(launch(decode::nvfp4_gemm_decode_split_kernel<T>, grid * decode::kSplit,
+                                      decode::THREADS, decode::SplitCfg<T>::SMEM_ALLOC, stream, true, tw, tx, p));
+        }
+    }
     return cuda_status(launch(decode::nvfp4_gemm_decode_kernel<T>, grid, decode::THREADS, decode::Cfg<T>::SMEM_ALLOC,
                               stream, true, tw, tx, p));
 }

@@ -103,3 +103,33 @@ def test_decode_gemm_late_stall_is_reported(nv, m):
     ref = oracle.linear_reference(xb, wb, off)
     assert_gemm_close(y.cpu().numpy(), ref["y"], bf16=False)
 
+
+
+@pytest.mark.parametrize("late", [False, True], ids=["second_stage", "last_stage"])
+def test_split_k_decode_stall_is_reported_and_the_context_stays_usable(nv, late):
+    """The split-K decode GEMM (8 tokens, N = 512: one cluster of four CTAs,
+    each on a quarter of K) withholds a stage in every CTA: the waits run out,
+    the three CTAs still push their (zero) partial sums so that CTA 0's slot
+    barrier completes, and the same context then computes the right answer."""
+    import torch
+    m, n, k = 8, 512, 2048
+    xb, wb, off = W.random_case(81, m, n, k)
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    qx, sfx, sx = nv.quantize_act(x)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    stall = nv.FLAG_TEST_STALL_LATE if late else nv.FLAG_TEST_STALL
+    nv.set_wait_timeout_ns(2_000_000)
+    try:
+        for _ in range(2):
+            nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT | stall)
+            assert nv.get_device_error() == nv.ERR_TIMEOUT
+            assert nv.get_device_error() == nv.OK
+    finally:
+        nv.set_wait_timeout_ns(2_000_000_000)
+    y = nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    ref = oracle.linear_reference(xb, wb, off)
+    assert_gemm_close(y.cpu().numpy(), ref["y"], bf16=False)

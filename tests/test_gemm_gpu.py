@@ -416,3 +416,35 @@ def test_static_weights_flag_changes_nothing_but_the_launch_order(nv, m):
         assert torch.equal(got[0], ref1) and torch.equal(got[2], ref1)
         assert torch.equal(got[1], ref2) and torch.equal(got[3], ref2)
 
+
+
+# Up to 16 tokens on few weight tiles (N up to 74 x 128) with K of at least 8
+# stages: the decode GEMM splits K over a cluster of four CTAs and reduces the
+# partial sums in CTA 0.  The down-projection of the decode workloads' model
+# (5120 x 17408), a ragged N with three modules, a partial last K stage.
+SPLIT_K_CASES = [
+    (1, 512, 2048, None),
+    (8, 1000, 5120, [264, 256, 480]),
+    (16, 5120, 17408, None),
+    (3, 2048, 2112, [1024, 1024]),
+    (12, 9472, 2048, None),
+]
+
+
+@pytest.mark.parametrize("m,n,k,segs", SPLIT_K_CASES)
+def test_split_k_decode_gemm(nv, m, n, k, segs):
+    import torch
+    xb, wb, off = W.random_case(500 + m, m, n, k, seg_rows=segs)
+    x = to_cuda_bf16(xb)
+    pw = nv.pack_weight(to_cuda_bf16(wb), off)
+    y32 = nv.linear_fused(x, pw, flags=nv.FLAG_F32_OUT)
+    ybf = nv.linear_fused(x, pw)
+    qx, sfx, sx = nv.quantize_act(x)
+    g32 = nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT)
+    gst = nv.gemm(qx, sfx, sx, m, pw, flags=nv.FLAG_F32_OUT | nv.FLAG_STATIC_WEIGHTS)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == nv.OK
+    ref = oracle.linear_reference(xb, wb, off)
+    assert_gemm_close(y32.cpu().numpy(), ref["y"], bf16=False)
+    assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), bf16_rne_from_f32(y32.cpu().numpy()))
+    assert torch.equal(y32, g32) and torch.equal(y32, gst)        # deterministic: the same sums in the same order
