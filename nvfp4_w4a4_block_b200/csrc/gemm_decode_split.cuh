@@ -15,7 +15,7 @@
 //   * CTA 0 adds them to its own in a fixed order (deterministic), scales by
 //     alpha(n) and stores, as the decode epilogue does.
 //
-// Used for up to 16 tokens; the kernel is otherwise the decode kernel's
+// Used for up to 32 tokens; the kernel is otherwise the decode kernel's
 // (programmatic dependent launch, early weight stages behind the library's
 // quantizer or with NVFP4_FLAG_STATIC_WEIGHTS, bounded waits, testing hooks).
 #pragma once
@@ -31,27 +31,30 @@ namespace nvfp4 {
 namespace decode {
 
 constexpr int kSplit = 4;
-constexpr int kSplitStages = 3;
 
 template <int T>
 struct SplitCfg {
+    // Three ring stages up to 16 tokens; at 32 the three partial slots (16 KB
+    // each) leave room for two beside them under two CTAs per SM.
+    static constexpr int STAGES = T <= 16 ? 3 : 2;
     static constexpr int B_BYTES = T * BK / 2;
     static constexpr int STAGE = A_BYTES + B_BYTES + 2 * SF_BYTES;
     static constexpr int SLOT = BW * T * 4;                       // one CTA's fp32 partial sums
     static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + kSplitStages * A_BYTES;
-    static constexpr int OFF_SFA = OFF_B + kSplitStages * B_BYTES;
-    static constexpr int OFF_SFB = OFF_SFA + kSplitStages * SF_BYTES;
-    static constexpr int OFF_SLOT = OFF_SFB + kSplitStages * SF_BYTES;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SF_BYTES;
+    static constexpr int OFF_SLOT = OFF_SFB + STAGES * SF_BYTES;
     static constexpr int OFF_BAR = OFF_SLOT + (kSplit - 1) * SLOT;
-    static constexpr int OFF_MISC = OFF_BAR + (2 * kSplitStages + 3) * 8;
+    static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 3) * 8;
     static constexpr int SMEM_ALLOC = OFF_MISC + 64 + 1024;
     static constexpr int TMEM_SFA = T;
     static constexpr int TMEM_SFB = T + KB * 4;
     static constexpr int TMEM_COLS = (T + KB * 8 <= 32) ? 32 : 64;
-    static_assert(T <= 16, "partials of more tokens do not fit beside the ring");
+    static_assert(T <= 32, "partials of more tokens do not fit beside the ring");
     static_assert(SMEM_ALLOC <= SMEM_LIMIT, "two CTAs per SM");
-    static_assert(kSplitStages * A_BYTES >= T * BW * 4, "the epilogue stages a fp32 tile in the weight buffers");
+    static_assert(STAGES * A_BYTES >= T * BW * 4, "the epilogue stages a fp32 tile in the weight buffers");
+    static_assert(TMEM_COLS >= T + KB * 8, "accumulator and scale columns");
     static_assert(SLOT % 16 == 0 && OFF_SLOT % 16 == 0, "16-byte partial pushes");
 };
 
@@ -73,8 +76,8 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(THREADS, 2)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *empty = full + kSplitStages;
-    uint64_t *acc_full = full + 2 * kSplitStages;
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *acc_full = full + 2 * C::STAGES;
     uint64_t *final_bar = acc_full + 1;
     uint64_t *slots_full = acc_full + 2;                          // CTA 0: every peer's partials landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
@@ -89,7 +92,7 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(THREADS, 2)
     const int nst = (static_cast<int>(rank) + 1) * p.k_stages / kSplit - ks_lo;   // >= 1: k_stages >= kSplit
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kSplitStages; ++s) {
+        for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -115,7 +118,7 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(THREADS, 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        const int pre = min(kSplitStages, nst);
+        const int pre = min(C::STAGES, nst);
         if (!p.early_weights)
             pdl_wait_prerequisites();
         for (int j = 0; j < pre; ++j) {
@@ -140,8 +143,8 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(THREADS, 2)
             }
             __syncwarp();
         }
-        int stage = pre % kSplitStages;
-        uint32_t phase = (pre == kSplitStages) ? 1u : 0u;
+        int stage = pre % C::STAGES;
+        uint32_t phase = (pre == C::STAGES) ? 1u : 0u;
         int issued = pre;
         for (int j = pre; j < nst; ++j) {
             if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)))
@@ -159,19 +162,19 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(THREADS, 2)
             }
             __syncwarp();
             issued = j + 1;
-            if (++stage == kSplitStages) {
+            if (++stage == C::STAGES) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
         pdl_launch_dependents();
-        for (int q = 0; q < min(kSplitStages, issued); ++q) {
+        for (int q = 0; q < min(C::STAGES, issued); ++q) {
             const int j = issued - 1 - q;
             if (j == p.stall_stage)
                 continue;
             volatile int no_abort = 0;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[j % kSplitStages],
-                                                           static_cast<uint32_t>((j / kSplitStages) & 1), &no_abort,
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[j % C::STAGES],
+                                                           static_cast<uint32_t>((j / C::STAGES) & 1), &no_abort,
                                                            DRAIN_TIMEOUT_NS)))
                 *abort_flag = 1;
         }
@@ -206,7 +209,7 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(THREADS, 2)
                 tc_commit(&empty[stage]);
             }
             __syncwarp();
-            if (++stage == kSplitStages) {
+            if (++stage == C::STAGES) {
                 stage = 0;
                 phase ^= 1u;
             }

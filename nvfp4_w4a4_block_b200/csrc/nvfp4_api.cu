@@ -176,6 +176,9 @@ nvfp4_status device_setup(int *sms)
             cudaFuncSetAttribute(decode::nvfp4_gemm_decode_split_kernel<16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, decode::SplitCfg<16>::SMEM_ALLOC) !=
                 cudaSuccess ||
+            cudaFuncSetAttribute(decode::nvfp4_gemm_decode_split_kernel<32>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, decode::SplitCfg<32>::SMEM_ALLOC) !=
+                cudaSuccess ||
             cudaFuncSetAttribute(peak::mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  peak::SMEM_ALLOC) != cudaSuccess)
             return NVFP4_ERR_CUDA;
@@ -527,10 +530,10 @@ nvfp4_status launch_decode(const uint8_t *qx, const uint8_t *sfx, const float *s
     p.stall_stage = (flags & NVFP4_FLAG_TEST_STALL) ? 1 : (flags & NVFP4_FLAG_TEST_STALL_LATE) ? p.k_stages - 1 : -1;
     p.early_weights = early_weights ? 1 : 0;
     const int grid = static_cast<int>((n + decode::BW - 1) / decode::BW);
-    if constexpr (T <= 16) {
-        // Few weight tiles (at most one per two SMs) and a K of at least 8
-        // stages: each tile runs on a cluster of decode::kSplit CTAs, one K
-        // range each (gemm_decode_split.cuh).
+    if constexpr (T <= 32) {
+        // Up to 32 tokens, few weight tiles (at most one per two SMs) and a K
+        // of at least 8 stages: each tile runs on a cluster of decode::kSplit
+        // CTAs, one K range each (gemm_decode_split.cuh).
         if (grid * 2 <= kSplitMaxTilesTimes2 && p.k_stages >= 2 * decode::kSplit) {
             if (flags & NVFP4_FLAG_TEST_STALL_LATE)          // the last stage of each CTA's K range
                 p.stall_stage = p.k_stages / decode::kSplit - 1;

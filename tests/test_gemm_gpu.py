@@ -418,7 +418,7 @@ def test_static_weights_flag_changes_nothing_but_the_launch_order(nv, m):
 
 
 
-# Up to 16 tokens on few weight tiles (N up to 74 x 128) with K of at least 8
+# Up to 32 tokens on few weight tiles (N up to 74 x 128) with K of at least 8
 # stages: the decode GEMM splits K over a cluster of four CTAs and reduces the
 # partial sums in CTA 0.  The down-projection of the decode workloads' model
 # (5120 x 17408), a ragged N with three modules, a partial last K stage.
@@ -428,6 +428,8 @@ SPLIT_K_CASES = [
     (16, 5120, 17408, None),
     (3, 2048, 2112, [1024, 1024]),
     (12, 9472, 2048, None),
+    (32, 5120, 17408, None),
+    (24, 1000, 2112, [264, 256, 480]),
 ]
 
 
